@@ -1,0 +1,371 @@
+// lynx_api.cu -- the C ABI of include/lynx.h: argument checks, workspace
+// layout, TMA descriptor encoding, kernel launches, device status and the
+// host-side metadata layout conversions.
+#include <cudaTypedefs.h>
+
+#include <atomic>
+#include <cstring>
+#include <mutex>
+
+#include "lynx.h"
+#include "lynx_internal.h"
+
+// Per-device status word: the first error code a kernel records wins.
+static __device__ uint32_t g_lynx_status_word;
+
+namespace lynx {
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+std::atomic<int> g_stall{0};
+
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+
+struct DeviceState {
+  std::once_flag once;
+  uint32_t* status = nullptr;
+  int sms = 0;
+  cudaError_t err = cudaSuccess;
+};
+DeviceState g_dev[kMaxDevices];
+
+void resolve_encode() {
+  void* fn = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+      q == cudaDriverEntryPointSuccess)
+    g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+}
+
+// Current device's state (status word address, SM count), set up once.
+DeviceState* device_state() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  DeviceState& d = g_dev[dev];
+  std::call_once(d.once, [&d, dev]() {
+    void* p = nullptr;
+    d.err = cudaGetSymbolAddress(&p, g_lynx_status_word);
+    if (d.err == cudaSuccess) d.status = static_cast<uint32_t*>(p);
+    if (d.err == cudaSuccess) d.err = cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev);
+  });
+  return d.err == cudaSuccess ? &d : nullptr;
+}
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+inline size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+struct WorkspaceLayout {
+  size_t vals, meta, scale, t, total;
+};
+
+WorkspaceLayout workspace_layout(int64_t M, int64_t K, int64_t r) {
+  WorkspaceLayout w;
+  w.vals = 0;
+  w.meta = align256(w.vals + static_cast<size_t>(M) * static_cast<size_t>(K));
+  w.scale = align256(w.meta + lynx_meta_bytes(M, K));
+  w.t = align256(w.scale + static_cast<size_t>(M) * 4);
+  w.total = align256(w.t + static_cast<size_t>(M) * static_cast<size_t>(r > 0 ? r : kLoraRank) * 2);
+  return w;
+}
+
+lynx_status check_shape(int64_t M, int64_t N, int64_t K) {
+  if (M < 1 || K < 64 || K % 64 != 0) return LYNX_ERR_UNSUPPORTED_SHAPE;
+  if (N != 0 && (N < 8 || N % 8 != 0)) return LYNX_ERR_UNSUPPORTED_SHAPE;
+  // TMA coordinates are 32-bit; keep every extent comfortably inside
+  if (M > (int64_t(1) << 30) || K > (int64_t(1) << 30) || N > (int64_t(1) << 30))
+    return LYNX_ERR_UNSUPPORTED_SHAPE;
+  return LYNX_OK;
+}
+
+lynx_status check_lora(const void* A, const void* B, int64_t r) {
+  if ((A == nullptr) != (B == nullptr)) return LYNX_ERR_INVALID_ARG;
+  if (A != nullptr && r != kLoraRank) return LYNX_ERR_UNSUPPORTED_SHAPE;
+  if (A == nullptr && r != 0 && r != kLoraRank) return LYNX_ERR_UNSUPPORTED_SHAPE;
+  return LYNX_OK;
+}
+
+lynx_status map_cuda(cudaError_t e) { return e == cudaSuccess ? LYNX_OK : LYNX_ERR_CUDA; }
+
+int gemm_bn(int64_t N) { return N >= 1024 ? 256 : 128; }
+
+lynx_status run_sparsify(DeviceState* ds, const void* X, const void* A, int64_t M, int64_t K,
+                         void* vals, void* meta, float* row_scale, void* t_out, int mode,
+                         cudaStream_t stream) {
+  SparsifyLaunch p;
+  std::memset(&p, 0, sizeof(p));
+  if (!encode_bf16_2d(&p.tm_x, X, K, M, K * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B))
+    return LYNX_ERR_CUDA;
+  if (mode & kModeLora) {
+    if (!encode_bf16_2d(&p.tm_a, A, K, kLoraRank, K * 2, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B))
+      return LYNX_ERR_CUDA;
+  }
+  p.vals = vals;
+  p.meta = static_cast<uint8_t*>(meta);
+  p.row_scale = row_scale;
+  p.t_out = t_out;
+  p.M = M;
+  p.K = K;
+  p.mode = mode;
+  p.cluster = (mode & kModeSelect) ? choose_sparsify_cluster(M, K, ds->sms)
+                                   : choose_sparsify_cluster(M, K, ds->sms);
+  p.boxes_per_cta = static_cast<int>(K / 64 / p.cluster);
+  p.kblocks = static_cast<int>((K + 127) / 128);
+  p.stall_test = g_stall.load();
+  p.status = ds->status;
+  return map_cuda(launch_sparsify(p, stream));
+}
+
+lynx_status run_gemm(DeviceState* ds, const void* a_src, bool sparse, const void* meta,
+                     const void* T, const void* W, const void* bias, const void* B, int64_t M,
+                     int64_t N, int64_t K, void* Y, cudaStream_t stream) {
+  GemmLaunch p;
+  std::memset(&p, 0, sizeof(p));
+  const int bn = gemm_bn(N);
+  if (sparse) {
+    if (!encode_bf16_2d(&p.tm_a, a_src, K / 2, M, K, 32, 128, CU_TENSOR_MAP_SWIZZLE_64B))
+      return LYNX_ERR_CUDA;
+  } else {
+    if (!encode_bf16_2d(&p.tm_a, a_src, K, M, K * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B))
+      return LYNX_ERR_CUDA;
+  }
+  if (!encode_bf16_2d(&p.tm_b, W, K, N, K * 2, 64, bn, CU_TENSOR_MAP_SWIZZLE_128B))
+    return LYNX_ERR_CUDA;
+  const bool lora = (T != nullptr && B != nullptr);
+  if (lora) {
+    if (!encode_bf16_2d(&p.tm_t, T, kLoraRank, M, kLoraRank * 2, 32, 128, CU_TENSOR_MAP_SWIZZLE_64B))
+      return LYNX_ERR_CUDA;
+    if (!encode_bf16_2d(&p.tm_lb, B, kLoraRank, N, kLoraRank * 2, 32, bn, CU_TENSOR_MAP_SWIZZLE_64B))
+      return LYNX_ERR_CUDA;
+  }
+  p.meta = static_cast<const uint8_t*>(meta);
+  p.bias = bias;
+  p.y = Y;
+  p.M = M;
+  p.N = N;
+  p.K = K;
+  p.sparse = sparse ? 1 : 0;
+  p.lora = lora ? 1 : 0;
+  p.bn = bn;
+  const int64_t tiles = ((M + 127) / 128) * ((N + bn - 1) / bn);
+  p.grid = static_cast<int>(tiles < ds->sms ? tiles : ds->sms);
+  p.stall_test = g_stall.load();
+  p.status = ds->status;
+  return map_cuda(launch_gemm(p, stream));
+}
+
+}  // namespace
+
+bool encode_bf16_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer,
+                    uint64_t row_pitch_bytes, uint32_t box_inner, uint32_t box_outer,
+                    CUtensorMapSwizzle swizzle) {
+  std::call_once(g_encode_once, resolve_encode);
+  if (g_encode == nullptr) return false;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {row_pitch_bytes};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
+                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+int device_sm_count() {
+  DeviceState* d = device_state();
+  return d ? d->sms : 0;
+}
+
+}  // namespace lynx
+
+using namespace lynx;
+
+extern "C" {
+
+const char* lynx_status_string(int status) {
+  switch (status) {
+    case LYNX_OK: return "LYNX_OK";
+    case LYNX_ERR_INVALID_ARG: return "LYNX_ERR_INVALID_ARG";
+    case LYNX_ERR_UNSUPPORTED_SHAPE: return "LYNX_ERR_UNSUPPORTED_SHAPE";
+    case LYNX_ERR_MISALIGNED: return "LYNX_ERR_MISALIGNED";
+    case LYNX_ERR_WORKSPACE_TOO_SMALL: return "LYNX_ERR_WORKSPACE_TOO_SMALL";
+    case LYNX_ERR_CUDA: return "LYNX_ERR_CUDA";
+    case LYNX_ERR_DEVICE_TIMEOUT: return "LYNX_ERR_DEVICE_TIMEOUT";
+    default: return "LYNX_ERR_UNKNOWN";
+  }
+}
+
+int lynx_version(void) { return (1 << 16) | 0; }
+
+int lynx_lora_rank(void) { return kLoraRank; }
+
+size_t lynx_vals_bytes(int64_t M, int64_t K) {
+  if (M < 0 || K < 0) return 0;
+  return static_cast<size_t>(M) * static_cast<size_t>(K);
+}
+
+size_t lynx_meta_bytes(int64_t M, int64_t K) {
+  if (M <= 0 || K <= 0) return 0;
+  return static_cast<size_t>((M + 127) / 128) * static_cast<size_t>((K + 127) / 128) *
+         static_cast<size_t>(kMetaBlockBytes);
+}
+
+size_t lynx_workspace_bytes(int64_t M, int64_t N, int64_t K, int64_t r) {
+  (void)N;
+  if (M <= 0 || K <= 0) return 0;
+  return workspace_layout(M, K, r).total;
+}
+
+int lynx_sparsify(const void* X, int64_t M, int64_t K, void* vals, void* meta, float* row_scale,
+                  void* stream) {
+  if (X == nullptr || vals == nullptr || meta == nullptr) return LYNX_ERR_INVALID_ARG;
+  lynx_status st = check_shape(M, 0, K);
+  if (st != LYNX_OK) return st;
+  if (!aligned16(X) || !aligned16(vals) || !aligned16(meta) ||
+      (reinterpret_cast<uintptr_t>(row_scale) & 3u) != 0)
+    return LYNX_ERR_MISALIGNED;
+  DeviceState* ds = device_state();
+  if (ds == nullptr) return LYNX_ERR_CUDA;
+  return run_sparsify(ds, X, nullptr, M, K, vals, meta, row_scale, nullptr, kModeSelect,
+                      static_cast<cudaStream_t>(stream));
+}
+
+int lynx_linear(const void* X, const void* W, const void* bias, const void* A, const void* B,
+                int64_t M, int64_t N, int64_t K, int64_t r, int skip_sparsify, void* Y,
+                void* workspace, size_t workspace_bytes, void* stream) {
+  if (X == nullptr || W == nullptr || Y == nullptr) return LYNX_ERR_INVALID_ARG;
+  lynx_status st = check_lora(A, B, r);
+  if (st != LYNX_OK) return st;
+  st = check_shape(M, N, K);
+  if (st != LYNX_OK) return st;
+  if (!aligned16(X) || !aligned16(W) || !aligned16(Y) || (bias && !aligned16(bias)) ||
+      (A && !aligned16(A)) || (B && !aligned16(B)) || (workspace && !aligned16(workspace)))
+    return LYNX_ERR_MISALIGNED;
+  const bool lora = A != nullptr;
+  const bool need_ws = lora || !skip_sparsify;
+  const WorkspaceLayout wl = workspace_layout(M, K, r);
+  if (need_ws && (workspace == nullptr || workspace_bytes < wl.total))
+    return workspace == nullptr ? LYNX_ERR_INVALID_ARG : LYNX_ERR_WORKSPACE_TOO_SMALL;
+  DeviceState* ds = device_state();
+  if (ds == nullptr) return LYNX_ERR_CUDA;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  void* t_buf = lora ? ws + wl.t : nullptr;
+  if (!skip_sparsify) {
+    st = run_sparsify(ds, X, A, M, K, ws + wl.vals, ws + wl.meta,
+                      reinterpret_cast<float*>(ws + wl.scale), t_buf,
+                      kModeSelect | (lora ? kModeLora : 0), s);
+    if (st != LYNX_OK) return st;
+    return run_gemm(ds, ws + wl.vals, true, ws + wl.meta, t_buf, W, bias, B, M, N, K, Y, s);
+  }
+  if (lora) {
+    st = run_sparsify(ds, X, A, M, K, nullptr, nullptr, nullptr, t_buf, kModeLora, s);
+    if (st != LYNX_OK) return st;
+  }
+  return run_gemm(ds, X, false, nullptr, t_buf, W, bias, B, M, N, K, Y, s);
+}
+
+int lynx_linear_dense(const void* X, const void* W, const void* bias, const void* A,
+                      const void* B, int64_t M, int64_t N, int64_t K, int64_t r, void* Y,
+                      void* workspace, size_t workspace_bytes, void* stream) {
+  return lynx_linear(X, W, bias, A, B, M, N, K, r, 1, Y, workspace, workspace_bytes, stream);
+}
+
+int lynx_sparse_gemm(const void* vals, const void* meta, const void* T, const void* W,
+                     const void* bias, const void* B, int64_t M, int64_t N, int64_t K, int64_t r,
+                     void* Y, void* stream) {
+  if (vals == nullptr || meta == nullptr || W == nullptr || Y == nullptr) return LYNX_ERR_INVALID_ARG;
+  lynx_status st = check_lora(T, B, r);
+  if (st != LYNX_OK) return st;
+  st = check_shape(M, N, K);
+  if (st != LYNX_OK) return st;
+  if (!aligned16(vals) || !aligned16(meta) || !aligned16(W) || !aligned16(Y) ||
+      (bias && !aligned16(bias)) || (T && !aligned16(T)) || (B && !aligned16(B)))
+    return LYNX_ERR_MISALIGNED;
+  DeviceState* ds = device_state();
+  if (ds == nullptr) return LYNX_ERR_CUDA;
+  return run_gemm(ds, vals, true, meta, T, W, bias, B, M, N, K, Y, static_cast<cudaStream_t>(stream));
+}
+
+int lynx_check_error(void* stream, uint32_t* device_code) {
+  if (device_code) *device_code = 0;
+  DeviceState* ds = device_state();
+  if (ds == nullptr) return LYNX_ERR_CUDA;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return LYNX_ERR_CUDA;
+  uint32_t code = 0;
+  e = cudaMemcpyFromSymbolAsync(&code, g_lynx_status_word, sizeof(code), 0, cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return LYNX_ERR_CUDA;
+  if (code != 0) {
+    const uint32_t zero = 0;
+    e = cudaMemcpyToSymbolAsync(g_lynx_status_word, &zero, sizeof(zero), 0, cudaMemcpyHostToDevice, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return LYNX_ERR_CUDA;
+  }
+  if (device_code) *device_code = code;
+  return code != 0 ? LYNX_ERR_DEVICE_TIMEOUT : LYNX_OK;
+}
+
+// hardware position of (row m, dense column k) inside the metadata buffer:
+// byte offset and the shift of the group's nibble inside that byte
+static inline void meta_hw_position(int64_t m, int64_t k, int64_t kblocks, size_t* byte,
+                                    int* shift) {
+  const int64_t mb = m / 128, kb = k / 128;
+  const int64_t mi = m % 128, ki = k % 128;
+  const int64_t lane = (mi % 8) + 8 * ((ki / 16) % 2) + 16 * (mi / 16);
+  const int64_t word = ki / 32;
+  const int64_t bit = (ki % 16) + 16 * ((mi / 8) % 2);
+  *byte = static_cast<size_t>((mb * kblocks + kb) * 2048 + lane * 16 + word * 4 + bit / 8);
+  *shift = static_cast<int>(bit % 8);
+}
+
+int lynx_meta_hw_to_canonical(const uint8_t* hw, uint8_t* canonical, int64_t M, int64_t K) {
+  if (hw == nullptr || canonical == nullptr) return LYNX_ERR_INVALID_ARG;
+  if (M < 1 || K < 8 || K % 8 != 0) return LYNX_ERR_UNSUPPORTED_SHAPE;
+  const int64_t kblocks = (K + 127) / 128;
+  for (int64_t m = 0; m < M; ++m) {
+    for (int64_t g = 0; g < K / 4; ++g) {
+      size_t byte;
+      int shift;
+      meta_hw_position(m, 4 * g, kblocks, &byte, &shift);
+      const uint8_t nib = static_cast<uint8_t>((hw[byte] >> shift) & 0xF);
+      uint8_t& dst = canonical[m * (K / 8) + g / 2];
+      if (g % 2 == 0)
+        dst = nib;
+      else
+        dst = static_cast<uint8_t>(dst | (nib << 4));
+    }
+  }
+  return LYNX_OK;
+}
+
+int lynx_meta_canonical_to_hw(const uint8_t* canonical, uint8_t* hw, int64_t M, int64_t K) {
+  if (hw == nullptr || canonical == nullptr) return LYNX_ERR_INVALID_ARG;
+  if (M < 1 || K < 8 || K % 8 != 0) return LYNX_ERR_UNSUPPORTED_SHAPE;
+  const int64_t kblocks = (K + 127) / 128;
+  const int64_t mpad = (M + 127) / 128 * 128;
+  std::memset(hw, 0, lynx_meta_bytes(M, K));
+  for (int64_t m = 0; m < mpad; ++m) {
+    for (int64_t g = 0; g < K / 4; ++g) {
+      uint8_t nib = 0x4;  // positions 0,1: the pattern of an all-zero group
+      if (m < M) {
+        const uint8_t b = canonical[m * (K / 8) + g / 2];
+        nib = static_cast<uint8_t>((g % 2 == 0) ? (b & 0xF) : (b >> 4));
+      }
+      size_t byte;
+      int shift;
+      meta_hw_position(m, 4 * g, kblocks, &byte, &shift);
+      hw[byte] = static_cast<uint8_t>(hw[byte] | (nib << shift));
+    }
+  }
+  return LYNX_OK;
+}
+
+int lynx_debug_set_stall(int enable) { return g_stall.exchange(enable ? 1 : 0); }
+
+}  // extern "C"

@@ -1,0 +1,69 @@
+// lynx_internal.h -- declarations shared by the library's translation units.
+// Not part of the public ABI (that is include/lynx.h).
+#pragma once
+
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+namespace lynx {
+
+constexpr int kLoraRank = 64;       // r: the only LoRA rank the kernels are built for
+constexpr int kRowBlock = 128;      // rows per metadata block / per MMA tile
+constexpr int kMetaBlockK = 128;    // dense K per metadata block
+constexpr int kMetaBlockBytes = 2048;  // 128 TMEM lanes x 16 bytes
+
+// ---- sparsify / LoRA-down pass ---------------------------------------------
+
+enum SparsifyMode : int { kModeSelect = 1, kModeLora = 2 };
+
+struct SparsifyLaunch {
+  CUtensorMap tm_x;     // X [M,K] bf16, box 64 x 128, 128B swizzle
+  CUtensorMap tm_a;     // A [64,K] bf16, box 64 x 64, 128B swizzle (mode & kModeLora)
+  void* vals;           // [M, K/2] bf16 (mode & kModeSelect)
+  uint8_t* meta;        // hardware-layout metadata blocks (mode & kModeSelect)
+  float* row_scale;     // [M] or null
+  void* t_out;          // [M, 64] bf16 (mode & kModeLora)
+  int64_t M, K;
+  int mode;
+  int cluster;          // CTAs per row block along K (1, 2, 4 or 8)
+  int boxes_per_cta;    // 64-column boxes each CTA covers
+  int kblocks;          // metadata blocks per row block: ceil(K/128)
+  int stall_test;       // test-only: the producer never loads, waits must time out
+  uint32_t* status;     // device status word (first error code wins)
+};
+
+cudaError_t launch_sparsify(const SparsifyLaunch& p, cudaStream_t stream);
+int choose_sparsify_cluster(int64_t M, int64_t K, int num_sms);
+
+// ---- tcgen05 GEMM with LoRA-up + bias epilogue ------------------------------
+
+struct GemmLaunch {
+  CUtensorMap tm_a;     // sparse: vals [M,K/2] box 32x128 SW64; dense: X [M,K] box 64x128 SW128
+  CUtensorMap tm_b;     // W [N,K] box 64 x BN, SW128
+  CUtensorMap tm_t;     // T [M,64] box 32 x 128, SW64 (lora)
+  CUtensorMap tm_lb;    // B [N,64] box 32 x BN, SW64 (lora)
+  const uint8_t* meta;  // hardware metadata blocks (sparse)
+  const void* bias;     // [N] bf16 or null
+  void* y;              // [M,N] bf16
+  int64_t M, N, K;
+  int sparse;
+  int lora;
+  int bn;               // 128 or 256
+  int grid;             // persistent CTAs
+  int stall_test;
+  uint32_t* status;
+};
+
+cudaError_t launch_gemm(const GemmLaunch& p, cudaStream_t stream);
+
+// ---- helpers ----------------------------------------------------------------
+
+// 2-D bf16 tensor map: inner (contiguous) extent, outer extent, row pitch in bytes
+bool encode_bf16_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer,
+                    uint64_t row_pitch_bytes, uint32_t box_inner, uint32_t box_outer,
+                    CUtensorMapSwizzle swizzle);
+
+int device_sm_count();
+
+}  // namespace lynx

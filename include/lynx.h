@@ -1,0 +1,162 @@
+/*
+ * lynx.h -- C ABI of the B200 (sm_100a) RT-Lynx online 2:4 activation-sparse
+ * linear layer.
+ *
+ * The layer (RT-Lynx pages; "qingkeai.online article" = the RT-Lynx article on
+ * qingkeai.online, "ai-feeds summary" = the ai-feeds.com summary of the paper):
+ *
+ *     Y = S(X) W^T + bias + (X A^T) B^T
+ *
+ *   - S(X): per token row, each group of 4 consecutive K-values keeps its 2
+ *     largest magnitudes, ties to the lower position (qingkeai.online article
+ *     section 02: Y = S(X) W^T with a 2:4 pattern made at run time; section 03:
+ *     Top-K).  The kept values are multiplied by the norm-compensation factor
+ *     s = sum|x| / sum|kept| of the row, computed in fp32 (section 03.1; ai-feeds
+ *     summary, core module 1), and rounded to bf16.
+ *   - (X A^T) B^T: LoRA residual of rank r = 64 on the dense X, frozen W
+ *     (section 03.2; neuraltrendhub summary: rank 64).
+ *   - skip_sparsify: the layer stays dense, S(X) = X (section 03.3, selective
+ *     layer skipping).
+ *   - The sparse product runs on sparse tensor cores (tcgen05.mma.sp) with the
+ *     compression, metadata layout, sparse GEMM and LoRA residual in CUDA
+ *     kernels of this library (section 04).
+ *
+ * Conventions for every entry point:
+ *   - Tensors are bf16 (IEEE binary16-brain, 2 bytes), row-major, contiguous,
+ *     given as plain device pointers.  The caller owns and allocates every
+ *     buffer; the library never allocates device memory.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *     Calls only enqueue work and return; nothing synchronises except
+ *     lynx_check_error.
+ *   - Return value: a lynx_status.  Host-side checks run before anything is
+ *     enqueued: on failure nothing is launched and no buffer is touched.
+ *     Device-side failures (a bounded wait that gave up) are recorded in a
+ *     per-device status word that lynx_check_error reports.
+ *   - Inputs must be finite; NaN/Inf inputs give unspecified (but memory-safe)
+ *     results.
+ *   - Shapes: M >= 1 tokens, K >= 64 with K % 64 == 0, N >= 8 with N % 8 == 0,
+ *     r = 64 when a LoRA branch is given.  Every pointer 16-byte aligned.
+ *   - Thread safety: calls from several host threads on different streams are
+ *     safe.  Calls whose device work overlaps must not share output buffers or
+ *     a workspace.
+ */
+#ifndef LYNX_H_
+#define LYNX_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define LYNX_API __attribute__((visibility("default")))
+#else
+#define LYNX_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum lynx_status {
+  LYNX_OK = 0,
+  LYNX_ERR_INVALID_ARG = 1,         /* null pointer, A without B, bad flag */
+  LYNX_ERR_UNSUPPORTED_SHAPE = 2,   /* M < 1, K % 64, N % 8, r != 64, ... */
+  LYNX_ERR_MISALIGNED = 3,          /* a pointer not 16-byte aligned */
+  LYNX_ERR_WORKSPACE_TOO_SMALL = 4, /* workspace_bytes < lynx_workspace_bytes() */
+  LYNX_ERR_CUDA = 5,                /* a CUDA runtime/driver call failed */
+  LYNX_ERR_DEVICE_TIMEOUT = 6       /* a kernel gave up a bounded wait */
+} lynx_status;
+
+/* Human-readable name of a status code (static storage, never NULL). */
+LYNX_API const char* lynx_status_string(int status);
+
+/* ABI version: (major << 16) | minor. */
+LYNX_API int lynx_version(void);
+
+/* Rank of the LoRA branch the kernels implement (64). */
+LYNX_API int lynx_lora_rank(void);
+
+/* ---- sizes ------------------------------------------------------------- */
+
+/* Bytes of the compressed values S(X): M x K/2 bf16 = M*K bytes. */
+LYNX_API size_t lynx_vals_bytes(int64_t M, int64_t K);
+
+/* Bytes of the 2:4 metadata in the tcgen05.mma.sp operand layout: one
+ * 2048-byte block per 128 rows x 128 dense K, rows padded to a multiple of 128
+ * and K to a multiple of 128: ceil(M/128) * ceil(K/128) * 2048.
+ * Layout: block (mb, kb) at byte (mb * ceil(K/128) + kb) * 2048; inside a
+ * block, row m and dense column k (both relative to the block) map to TMEM
+ * lane L = (m % 8) + 8 * ((k / 16) % 2) + 16 * (m / 16), 32-bit word
+ * w = k / 32 of the lane's 16 bytes, bit b = (k % 16) + 16 * ((m / 8) % 2);
+ * each group of 4 owns 4 bits: lo | hi << 2 (lo < hi its kept positions). */
+LYNX_API size_t lynx_meta_bytes(int64_t M, int64_t K);
+
+/* Bytes of the workspace lynx_linear needs (compressed values, metadata, row
+ * scales, the bf16 LoRA down-projection T [M,64], alignment padding). */
+LYNX_API size_t lynx_workspace_bytes(int64_t M, int64_t N, int64_t K, int64_t r);
+
+/* ---- the layer --------------------------------------------------------- */
+
+/* S(X) alone (qingkeai.online article sections 02-03.1; ai-feeds summary,
+ * core module 1).
+ *   X         [M,K] bf16, input activations (read only)
+ *   vals      [M,K/2] bf16, out: kept values after compensation, two per group,
+ *             ascending position (lynx_vals_bytes)
+ *   meta      out: metadata blocks, lynx_meta_bytes(M,K) bytes (layout above);
+ *             rows M..ceil(M/128)*128-1 hold the pattern of an all-zero row
+ *   row_scale [M] fp32, out: s per row, or NULL
+ * The vals buffer is also used as the pass's own scratch while it runs. */
+LYNX_API int lynx_sparsify(const void* X, int64_t M, int64_t K, void* vals, void* meta, float* row_scale,
+                  void* stream);
+
+/* Y = S(X) W^T + bias + (X A^T) B^T  (S(X) = X when skip_sparsify != 0).
+ *   X [M,K], W [N,K] (frozen backbone weight), bias [N] or NULL,
+ *   A [r,K] and B [N,r] (LoRA, both or neither; r must be 64), Y [M,N] out.
+ *   workspace: caller-allocated device buffer of workspace_bytes >=
+ *   lynx_workspace_bytes(M,N,K,r); after the call it holds S(X) (vals, meta,
+ *   row scales) and T = X A^T as bf16, in that order at 256-byte aligned
+ *   offsets.  Y is bf16(acc + bias) with acc accumulated in fp32. */
+LYNX_API int lynx_linear(const void* X, const void* W, const void* bias, const void* A, const void* B,
+                int64_t M, int64_t N, int64_t K, int64_t r, int skip_sparsify, void* Y,
+                void* workspace, size_t workspace_bytes, void* stream);
+
+/* The dense path of a layer that selective layer skipping leaves dense
+ * (qingkeai.online article section 03.3): Y = X W^T + bias + (X A^T) B^T.
+ * Same arguments and workspace as lynx_linear. */
+LYNX_API int lynx_linear_dense(const void* X, const void* W, const void* bias, const void* A,
+                      const void* B, int64_t M, int64_t N, int64_t K, int64_t r, void* Y,
+                      void* workspace, size_t workspace_bytes, void* stream);
+
+/* The sparse product on an S(X) made earlier by lynx_sparsify (or the
+ * workspace of lynx_linear):  Y = S(X) W^T + bias + T B^T.
+ *   vals [M,K/2] and meta as written by lynx_sparsify; T [M,r] bf16 or NULL,
+ *   B [N,r] or NULL (both or neither, r = 64); other arguments as above. */
+LYNX_API int lynx_sparse_gemm(const void* vals, const void* meta, const void* T, const void* W,
+                     const void* bias, const void* B, int64_t M, int64_t N, int64_t K, int64_t r,
+                     void* Y, void* stream);
+
+/* ---- errors and metadata conversion ----------------------------------- */
+
+/* Synchronises `stream`, then reports (and clears) the current device's status
+ * word: LYNX_ERR_DEVICE_TIMEOUT if a kernel gave up a bounded wait since the
+ * last check, LYNX_ERR_CUDA if the stream holds a CUDA error, else LYNX_OK.
+ * *device_code (may be NULL) receives the raw device code (0 if none). */
+LYNX_API int lynx_check_error(void* stream, uint32_t* device_code);
+
+/* Host-side conversions between the hardware metadata layout (above) and the
+ * canonical one: row m owns K/8 bytes, group g is the nibble lo | hi << 2 in
+ * byte m*K/8 + g/2, low nibble for even g.  Host pointers; K % 8 == 0.
+ * canonical_to_hw fills padding rows with the all-zero-row pattern (lo=0,hi=1)
+ * and padding K with zero bits. */
+LYNX_API int lynx_meta_hw_to_canonical(const uint8_t* hw, uint8_t* canonical, int64_t M, int64_t K);
+LYNX_API int lynx_meta_canonical_to_hw(const uint8_t* canonical, uint8_t* hw, int64_t M, int64_t K);
+
+/* Test hook (not for production use): when nonzero, kernels launched after
+ * this call never load their inputs, so their bounded waits run out (about 2 s)
+ * and lynx_check_error reports LYNX_ERR_DEVICE_TIMEOUT.  Returns the old value. */
+LYNX_API int lynx_debug_set_stall(int enable);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LYNX_H_ */

@@ -1,0 +1,271 @@
+"""Parity of the CUDA path (through the C ABI) with the CPU oracle.
+
+Bars (the layer's stated tolerances):
+  * metadata (kept positions) bit-exact, compared in the canonical layout;
+  * compressed values within 1 bf16 ulp (the fp32 row sums are added in a
+    different order on the GPU);
+  * Y: elementwise |dY| <= 2e-2 * ||S(X)_m||_2 * ||W_n||_2 and relative
+    Frobenius error <= 5e-3 (fp32 accumulation, one bf16 rounding).
+Inputs come from the seeded generators; expected values only from the oracle.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from activation_sparse_gemm_lynx_b200 import lynx, workloads
+
+import helpers
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda:0"
+
+
+def dev(bits):
+    if bits is None:
+        return None
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(DEV)
+
+
+def host(t):
+    return t.detach().contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    assert torch.cuda.is_available(), "these tests need a GPU"
+    torch.cuda.set_device(0)
+    lynx.library()
+    yield
+    st, code = lynx.lynx_check_error()
+    assert st == lynx.LYNX_OK, (st, code)
+
+
+def run_sparsify(X):
+    vals, meta, scale = lynx.lynx_sparsify(dev(X))
+    torch.cuda.synchronize()
+    return host(vals), meta.cpu().numpy(), scale.cpu().numpy()
+
+
+def check_sparsify(X, vals, meta, scale):
+    M, K = X.shape
+    ref = oracle.sparsify(X)
+    canon = helpers.canonical_from_hw(meta, M, K)
+    assert np.array_equal(canon, ref["meta"]), "metadata differs from the oracle"
+    # the library's own converter agrees with the test's reading of the layout
+    assert np.array_equal(lynx.lynx_meta_hw_to_canonical(meta, M, K), canon)
+    d = helpers.bf16_ulp_distance(vals, ref["vals"])
+    assert int(d.max()) <= 1, f"values differ by {int(d.max())} ulp"
+    assert np.allclose(scale, ref["scale"], rtol=4e-6, atol=0)
+    return ref
+
+
+# ---------------------------------------------------------------------------
+# S(X)
+
+
+def test_sparsify_tiny_config():
+    inp = workloads.make_config_inputs("tiny")
+    X = inp["X"]
+    check_sparsify(X, *run_sparsify(X))
+
+
+@pytest.mark.parametrize("M,K", [(1, 64), (130, 192), (300, 576), (257, 1024), (64, 3072),
+                                 (129, 12288)])
+def test_sparsify_shapes(M, K):
+    X = workloads.make_linear_inputs(M, K, 8, seed=M + K)["X"]
+    check_sparsify(X, *run_sparsify(X))
+
+
+def test_sparsify_ties_and_zeros():
+    rng = np.random.default_rng(3)
+    M, K = 192, 512
+    alphabet = np.array([0.0, -0.0, 1.0, -1.0, 2.0, -2.0, 0.5], dtype=np.float32)
+    x = alphabet[rng.integers(0, len(alphabet), size=(M, K))]
+    x[5] = 0.0                                        # an all-zero row: s = 1
+    X = workloads.f32_to_bf16_bits(x)
+    vals, meta, scale = run_sparsify(X)
+    check_sparsify(X, vals, meta, scale)
+    assert scale[5] == 1.0
+
+
+def test_sparsify_all_keep_is_identity():
+    rng = np.random.default_rng(4)
+    M, K = 130, 256
+    x = rng.standard_normal((M, K // 4, 4)).astype(np.float32)
+    for m in range(M):
+        for g in range(K // 4):
+            x[m, g, rng.choice(4, 2, replace=False)] = 0.0
+    X = workloads.f32_to_bf16_bits(x.reshape(M, K))
+    vals, meta, scale = run_sparsify(X)
+    check_sparsify(X, vals, meta, scale)
+    assert np.all(scale == 1.0)
+    dense = helpers.dense_from_canonical(vals, helpers.canonical_from_hw(meta, M, K), K)
+    assert np.array_equal(dense, helpers.f32(X).astype(np.float64))
+
+
+# ---------------------------------------------------------------------------
+# the sparse product alone, on an oracle-made S(X)
+
+
+@pytest.mark.parametrize("M,N,K", [(256, 512, 512), (200, 136, 576), (130, 1024, 256)])
+def test_sparse_gemm_on_oracle_sx(M, N, K):
+    inp = workloads.make_linear_inputs(M, K, N, seed=7)
+    ref = oracle.sparsify(inp["X"])
+    hw = helpers.hw_from_canonical(ref["meta"], M, K)
+    Y = lynx.lynx_sparse_gemm(dev(ref["vals"]), torch.from_numpy(hw).to(DEV), dev(inp["W"]),
+                              bias=dev(inp["bias"]))
+    y = helpers.f32(host(Y)).astype(np.float64)
+    SX = helpers.dense_from_canonical(ref["vals"], ref["meta"], K)
+    Wd = helpers.f32(inp["W"]).astype(np.float64)
+    y_ref = SX @ Wd.T + helpers.f32(inp["bias"]).astype(np.float64)
+    worst, fro = helpers.y_tolerance_check(y, y_ref, SX, Wd)
+    assert worst <= 1.0 and fro <= 5e-3, (worst, fro)
+
+
+def test_identity_weight_probe_pins_operand_layout():
+    """W = I: Y must reproduce S(X) exactly (each output is one exact product),
+    which pins the value and metadata layouts end to end."""
+    M, K = 256, 512
+    X = workloads.make_linear_inputs(M, K, 8, seed=31)["X"]
+    eye = workloads.f32_to_bf16_bits(np.eye(K, dtype=np.float32))
+    Y = lynx.lynx_linear(dev(X), dev(eye))
+    vals, meta, _ = run_sparsify(X)
+    dense = helpers.dense_from_canonical(vals, helpers.canonical_from_hw(meta, M, K), K)
+    y = helpers.f32(host(Y)).astype(np.float64)
+    assert np.array_equal(y, dense)
+    ref = oracle.sparsify(X)
+    ref_dense = helpers.dense_from_canonical(ref["vals"], ref["meta"], K)
+    assert np.array_equal(y != 0, ref_dense != 0)
+
+
+# ---------------------------------------------------------------------------
+# the whole layer
+
+
+def check_linear(inp, skip=False, rows=None):
+    X, W = inp["X"], inp["W"]
+    Y = lynx.lynx_linear(dev(X), dev(W), dev(inp["bias"]), dev(inp["A"]), dev(inp["B"]),
+                         skip_sparsify=skip)
+    torch.cuda.synchronize()
+    y = helpers.f32(host(Y)).astype(np.float64)
+    if rows is not None:
+        X = X[rows]
+        y = y[rows]
+    y_ref, _, sx = oracle.linear(X, W, inp["bias"], inp["A"], inp["B"], skip=skip, want_sx=True)
+    worst, fro = helpers.y_tolerance_check(y, y_ref, sx, helpers.f32(W).astype(np.float64))
+    assert worst <= 1.0 and fro <= 5e-3, (worst, fro)
+    return worst, fro
+
+
+def test_linear_tiny_config():
+    check_linear(workloads.make_config_inputs("tiny"))
+
+
+def test_linear_dense_path_tiny_config():
+    check_linear(workloads.make_config_inputs("tiny"), skip=True)
+
+
+@pytest.mark.parametrize("M,N,K,bias,lora", [
+    (300, 200, 576, True, True),     # ragged M and N, K % 128 == 64
+    (1, 8, 64, True, True),          # smallest shape
+    (129, 264, 1024, False, True),   # no bias
+    (256, 1024, 512, True, False),   # no LoRA, BN = 256
+    (200, 2048, 3072, True, True),   # cluster-split sparsify, several N tiles
+])
+def test_linear_shapes(M, N, K, bias, lora):
+    inp = workloads.make_linear_inputs(M, K, N, seed=M * 3 + N, bias=bias, lora=lora)
+    check_linear(inp)
+
+
+@pytest.mark.parametrize("M,N,K", [(300, 200, 576), (256, 1024, 512)])
+def test_linear_dense_shapes(M, N, K):
+    inp = workloads.make_linear_inputs(M, K, N, seed=11)
+    check_linear(inp, skip=True)
+
+
+def test_linear_is_deterministic():
+    inp = workloads.make_linear_inputs(384, 3072, 1024, seed=5)
+    args = [dev(inp[k]) for k in ("X", "W", "bias", "A", "B")]
+    y1 = host(lynx.lynx_linear(*args))
+    y2 = host(lynx.lynx_linear(*args))
+    assert np.array_equal(y1, y2)
+
+
+def test_workspace_holds_sx_and_t():
+    inp = workloads.make_linear_inputs(200, 576, 64, seed=17)
+    M, K = inp["X"].shape
+    ws = torch.zeros(lynx.lynx_workspace_bytes(M, 64, K, 64), dtype=torch.uint8, device=DEV)
+    lynx.lynx_linear(dev(inp["X"]), dev(inp["W"]), dev(inp["bias"]), dev(inp["A"]),
+                     dev(inp["B"]), workspace=ws)
+    torch.cuda.synchronize()
+    raw = ws.cpu().numpy()
+    vals = raw[: M * K].view(np.uint16).reshape(M, K // 2)
+    meta_off = (M * K + 255) // 256 * 256
+    meta = raw[meta_off: meta_off + lynx.lynx_meta_bytes(M, K)]
+    ref = oracle.sparsify(inp["X"])
+    assert np.array_equal(helpers.canonical_from_hw(meta, M, K), ref["meta"])
+    assert helpers.bf16_ulp_distance(vals, ref["vals"]).max() <= 1
+    t_off = (meta_off + lynx.lynx_meta_bytes(M, K) + 255) // 256 * 256
+    t_off = (t_off + 4 * M + 255) // 256 * 256
+    T = helpers.f32(raw[t_off: t_off + M * 128].view(np.uint16).reshape(M, 64)).astype(np.float64)
+    _, t_ref, _ = oracle.linear(inp["X"], inp["W"], inp["bias"], inp["A"], inp["B"])
+    # bf16 rounding of an fp32-accumulated dot product
+    assert np.all(np.abs(T - t_ref) <= 2 ** -8 * np.abs(t_ref) + 1e-6)
+
+
+# ---------------------------------------------------------------------------
+# full-size workloads, in the launch configuration the benchmark times: sampled
+# rows against the oracle (rows are independent)
+
+
+@pytest.mark.parametrize("name", ["attn_out", "mlp_up", "mlp_down"])
+def test_full_size_sampled_rows(name):
+    c = workloads.CONFIGS[name]
+    inp = workloads.make_config_inputs(name)
+    M, K = inp["X"].shape
+    rng = np.random.default_rng(99)
+    rows = np.unique(np.concatenate([[0, 127, 128, M - 1], rng.choice(M, 28, replace=False)]))
+    ws = torch.empty(lynx.lynx_workspace_bytes(M, c.N, K, 64), dtype=torch.uint8, device=DEV)
+    check_linear(inp, rows=rows)
+    # S(X) of the sampled rows, from the same kind of call
+    args = [dev(inp[k]) for k in ("X", "W", "bias", "A", "B")]
+    lynx.lynx_linear(*args, workspace=ws)
+    torch.cuda.synchronize()
+    raw = ws.cpu().numpy()
+    vals = raw[: M * K].view(np.uint16).reshape(M, K // 2)
+    meta_off = (M * K + 255) // 256 * 256
+    meta = raw[meta_off: meta_off + lynx.lynx_meta_bytes(M, K)]
+    canon = helpers.canonical_from_hw(meta, M, K)
+    ref = oracle.sparsify(inp["X"][rows])
+    assert np.array_equal(canon[rows], ref["meta"])
+    assert helpers.bf16_ulp_distance(vals[rows], ref["vals"]).max() <= 1
+
+
+# ---------------------------------------------------------------------------
+# errors
+
+
+def test_bad_workspace_is_rejected_before_launch():
+    inp = workloads.make_linear_inputs(128, 512, 256, seed=2)
+    ws = torch.empty(16, dtype=torch.uint8, device=DEV)
+    with pytest.raises(lynx.LynxError) as e:
+        lynx.lynx_linear(dev(inp["X"]), dev(inp["W"]), workspace=ws)
+    assert e.value.status == lynx.LYNX_ERR_WORKSPACE_TOO_SMALL
+
+
+def test_device_timeout_is_reported_and_context_survives():
+    X = workloads.make_linear_inputs(256, 512, 8, seed=1)["X"]
+    lynx.lynx_debug_set_stall(True)
+    try:
+        lynx.lynx_sparsify(dev(X))
+        st, code = lynx.lynx_check_error()
+    finally:
+        lynx.lynx_debug_set_stall(False)
+    assert st == lynx.LYNX_ERR_DEVICE_TIMEOUT
+    assert code != 0
+    st, code = lynx.lynx_check_error()
+    assert st == lynx.LYNX_OK and code == 0
+    # the context is still usable and the next call is correct
+    check_sparsify(X, *run_sparsify(X))
