@@ -22,8 +22,10 @@ from .lynx import (  # noqa: F401
     lynx_meta_bytes,
     lynx_meta_canonical_to_hw,
     lynx_meta_hw_to_canonical,
+    lynx_profile_set_split_event,
     lynx_sparse_gemm,
     lynx_sparsify,
+    lynx_sparsify_workspace_bytes,
     lynx_status_string,
     lynx_vals_bytes,
     lynx_version,

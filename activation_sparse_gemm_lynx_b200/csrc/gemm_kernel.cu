@@ -19,7 +19,8 @@
 //   warp 1      TMEM owner + MMA issuer (one thread): tcgen05.cp of metadata
 //               into a 4-slot TMEM ring, tcgen05.mma(.sp) into the accumulator,
 //               tcgen05.commit to release stages / publish the accumulator.
-//   warps 2-5   epilogue: tcgen05.ld 32x32b -> +bias -> bf16 -> global.
+//   warps 2-9   epilogue: tcgen05.ld 32x32b -> s * acc + bias -> bf16 -> global
+//               (two warps per TMEM lane quarter, half of the columns each).
 // Accumulators: 1 TMEM buffer for BN = 256, 2 (double buffered) for BN = 128.
 #include <cuda_bf16.h>
 
@@ -30,7 +31,7 @@ namespace lynx {
 
 namespace {
 
-constexpr int kGemmThreads = 192;
+constexpr int kGemmThreads = 320;  // producer, MMA, 8 epilogue warps
 constexpr uint32_t kTmemCols = 512;
 constexpr int kGroupM = 16;
 constexpr int kEslots = 4;
@@ -59,9 +60,13 @@ struct __align__(1024) GemmSmem {
   uint64_t acc_full[2];
   uint64_t acc_empty[2];
   uint64_t drain;
+  float bias_s[BN];  // the current tile's bias, fp32
   uint32_t tmem_base;
   volatile uint32_t abort_flag;
 };
+
+constexpr uint32_t kBarEpilogue = 2;  // named barrier of the 8 epilogue warps
+constexpr uint32_t kEpiThreads = 256;
 
 __device__ __forceinline__ void tile_coords(int tile, int ntm, int ntn, int& mb, int& nb) {
   const int per_group = kGroupM * ntn;
@@ -97,7 +102,7 @@ lynx_gemm_kernel(const __grid_constant__ GemmLaunch p) {
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&sm.acc_full[a], 1);
-      mbar_init(&sm.acc_empty[a], 4);
+      mbar_init(&sm.acc_empty[a], 8);
     }
     mbar_init(&sm.drain, 1);
     sm.abort_flag = 0u;
@@ -250,8 +255,14 @@ lynx_gemm_kernel(const __grid_constant__ GemmLaunch p) {
     __syncwarp();
   } else {
     // ------------------------------------------------------------ epilogue
-    const uint32_t q = warp & 3u;  // TMEM lane quarter this warp may access
+    // Y = bf16(s_row * acc + bias).  Two warps per TMEM lane quarter, each
+    // draining half of the columns into registers; the TMEM buffer is released
+    // before the global stores, so the next tile's MMAs overlap them.
+    constexpr int kHalf = BN / 2;
+    const uint32_t q = warp & 3u;              // TMEM lane quarter this warp may access
+    const uint32_t ch = (warp - 2u) >> 2;      // which half of the columns
     const uint32_t row = 32u * q + lane;
+    const uint32_t et = threadIdx.x - 64u;     // 0..255
     const __nv_bfloat16* bias = static_cast<const __nv_bfloat16*>(p.bias);
     __nv_bfloat16* y = static_cast<__nv_bfloat16*>(p.y);
     int acc_count = 0;
@@ -260,48 +271,52 @@ lynx_gemm_kernel(const __grid_constant__ GemmLaunch p) {
       tile_coords(tile, ntm, ntn, mb, nb);
       const int acc = acc_count % C::kAcc;
       const uint32_t acc_ph = static_cast<uint32_t>(acc_count / C::kAcc) & 1u;
-      if (sm.abort_flag || !mbar_wait(&sm.acc_full[acc], acc_ph)) {
-        if (!sm.abort_flag) {
-          record_error(p.status, kDevTimeoutAccum);
-          sm.abort_flag = 1u;
-        }
-        break;
-      }
-      tc_fence_after();
       const int64_t grow = static_cast<int64_t>(mb) * 128 + row;
       const bool row_ok = grow < p.M;
-      __nv_bfloat16* yrow = y + grow * p.N;
-#pragma unroll 1
-      for (int c = 0; c < BN / 32; ++c) {
+      const int64_t n_base = static_cast<int64_t>(nb) * BN;
+      named_bar_sync(kBarEpilogue, kEpiThreads);  // the previous tile's bias is no longer read
+      for (uint32_t j = et; j < static_cast<uint32_t>(BN); j += kEpiThreads) {
+        const int64_t n = n_base + j;
+        sm.bias_s[j] = (bias != nullptr && n < p.N) ? __bfloat162float(bias[n]) : 0.f;
+      }
+      const float s = (p.row_scale != nullptr && row_ok) ? p.row_scale[grow] : 1.f;
+      bool ok = !sm.abort_flag;
+      if (ok && !mbar_wait(&sm.acc_full[acc], acc_ph)) {
+        record_error(p.status, kDevTimeoutAccum);
+        sm.abort_flag = 1u;
+        ok = false;
+      }
+      // publishes the bias tile and makes the stop decision identical in all warps
+      if (named_bar_red_or(kBarEpilogue, kEpiThreads, !ok)) break;
+      tc_fence_after();
+      uint32_t out[kHalf / 2];
+#pragma unroll
+      for (int c = 0; c < kHalf / 32; ++c) {
+        const int col = static_cast<int>(ch) * kHalf + 32 * c;
         uint32_t r[32];
-        tmem_ld_32x32b_x32(sm.tmem_base + ((32u * q) << 16) + static_cast<uint32_t>(acc * BN + 32 * c), r);
+        tmem_ld_32x32b_x32(sm.tmem_base + ((32u * q) << 16) + static_cast<uint32_t>(acc * BN + col), r);
         tmem_ld_wait();
-        const int64_t n0 = static_cast<int64_t>(nb) * BN + 32 * c;
-        uint32_t out[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-          float a = __uint_as_float(r[2 * i]);
-          float b = __uint_as_float(r[2 * i + 1]);
-          if (bias != nullptr && n0 + 2 * i < p.N) {
-            const __nv_bfloat162 bb = *reinterpret_cast<const __nv_bfloat162*>(bias + n0 + 2 * i);
-            a = __fadd_rn(a, __bfloat162float(bb.x));
-            b = __fadd_rn(b, __bfloat162float(bb.y));
-          }
+          const float a = __fmaf_rn(s, __uint_as_float(r[2 * i]), sm.bias_s[col + 2 * i]);
+          const float b = __fmaf_rn(s, __uint_as_float(r[2 * i + 1]), sm.bias_s[col + 2 * i + 1]);
           __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
-          out[i] = *reinterpret_cast<uint32_t*>(&h);
-        }
-        if (row_ok) {
-#pragma unroll
-          for (int v = 0; v < 4; ++v) {
-            if (n0 + 8 * v < p.N)
-              *reinterpret_cast<uint4*>(yrow + n0 + 8 * v) =
-                  make_uint4(out[4 * v], out[4 * v + 1], out[4 * v + 2], out[4 * v + 3]);
-          }
+          out[16 * c + i] = *reinterpret_cast<uint32_t*>(&h);
         }
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.acc_empty[acc]);
+      if (row_ok) {
+        const int64_t n0 = n_base + static_cast<int64_t>(ch) * kHalf;
+        __nv_bfloat16* yrow = y + grow * p.N + n0;
+#pragma unroll
+        for (int v = 0; v < kHalf / 8; ++v) {
+          if (n0 + 8 * v < p.N)
+            *reinterpret_cast<uint4*>(yrow + 8 * v) =
+                make_uint4(out[4 * v], out[4 * v + 1], out[4 * v + 2], out[4 * v + 3]);
+        }
+      }
     }
   }
 

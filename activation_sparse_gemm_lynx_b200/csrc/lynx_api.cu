@@ -20,6 +20,7 @@ namespace {
 constexpr int kMaxDevices = 64;
 
 std::atomic<int> g_stall{0};
+std::atomic<void*> g_split_event{nullptr};
 
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 std::once_flag g_encode_once;
@@ -59,16 +60,35 @@ inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 
 inline size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
 struct WorkspaceLayout {
-  size_t vals, meta, scale, t, total;
+  size_t vals, meta, scale, t, lpart, tpart, total;
 };
 
+// lynx_linear's workspace: kept values | metadata | s | T (or T/s) | partials
 WorkspaceLayout workspace_layout(int64_t M, int64_t K, int64_t r) {
+  (void)r;
+  const size_t m = static_cast<size_t>(M);
   WorkspaceLayout w;
   w.vals = 0;
-  w.meta = align256(w.vals + static_cast<size_t>(M) * static_cast<size_t>(K));
+  w.meta = align256(w.vals + m * static_cast<size_t>(K));
   w.scale = align256(w.meta + lynx_meta_bytes(M, K));
-  w.t = align256(w.scale + static_cast<size_t>(M) * 4);
-  w.total = align256(w.t + static_cast<size_t>(M) * static_cast<size_t>(r > 0 ? r : kLoraRank) * 2);
+  w.t = align256(w.scale + m * 4);
+  w.lpart = align256(w.t + m * kLoraRank * 2);
+  w.tpart = align256(w.lpart + static_cast<size_t>(kMaxSplit) * m * 8);
+  w.total = align256(w.tpart + static_cast<size_t>(kMaxSplit) * m * kLoraRank * 4);
+  return w;
+}
+
+// lynx_sparsify's workspace: partial sums | s (used when no row_scale is given)
+struct SparsifyWorkspace {
+  size_t lpart, scale, total;
+};
+
+SparsifyWorkspace sparsify_workspace(int64_t M) {
+  const size_t m = static_cast<size_t>(M);
+  SparsifyWorkspace w;
+  w.lpart = 0;
+  w.scale = align256(static_cast<size_t>(kMaxSplit) * m * 8);
+  w.total = align256(w.scale + m * 4);
   return w;
 }
 
@@ -93,8 +113,8 @@ lynx_status map_cuda(cudaError_t e) { return e == cudaSuccess ? LYNX_OK : LYNX_E
 int gemm_bn(int64_t N) { return N >= 1024 ? 256 : 128; }
 
 lynx_status run_sparsify(DeviceState* ds, const void* X, const void* A, int64_t M, int64_t K,
-                         void* vals, void* meta, float* row_scale, void* t_out, int mode,
-                         cudaStream_t stream) {
+                         void* vals, void* meta, float* row_scale, void* t_out, float2* lpart,
+                         float* tpart, int mode, cudaStream_t stream) {
   SparsifyLaunch p;
   std::memset(&p, 0, sizeof(p));
   if (!encode_bf16_2d(&p.tm_x, X, K, M, K * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B))
@@ -103,16 +123,22 @@ lynx_status run_sparsify(DeviceState* ds, const void* X, const void* A, int64_t 
     if (!encode_bf16_2d(&p.tm_a, A, K, kLoraRank, K * 2, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B))
       return LYNX_ERR_CUDA;
   }
+  if (mode & kModeSelect) {
+    // kept values leave through TMA stores of 128 x 32 tiles
+    if (!encode_bf16_2d(&p.tm_vals, vals, K / 2, M, K, 32, 128, CU_TENSOR_MAP_SWIZZLE_64B))
+      return LYNX_ERR_CUDA;
+  }
   p.vals = vals;
   p.meta = static_cast<uint8_t*>(meta);
   p.row_scale = row_scale;
   p.t_out = t_out;
+  p.lpart = lpart;
+  p.tpart = tpart;
   p.M = M;
   p.K = K;
   p.mode = mode;
-  p.cluster = (mode & kModeSelect) ? choose_sparsify_cluster(M, K, ds->sms)
-                                   : choose_sparsify_cluster(M, K, ds->sms);
-  p.boxes_per_cta = static_cast<int>(K / 64 / p.cluster);
+  p.split = choose_sparsify_split(M, K, ds->sms);
+  p.boxes_per_cta = static_cast<int>(K / 64 / p.split);
   p.kblocks = static_cast<int>((K + 127) / 128);
   p.stall_test = g_stall.load();
   p.status = ds->status;
@@ -120,8 +146,8 @@ lynx_status run_sparsify(DeviceState* ds, const void* X, const void* A, int64_t 
 }
 
 lynx_status run_gemm(DeviceState* ds, const void* a_src, bool sparse, const void* meta,
-                     const void* T, const void* W, const void* bias, const void* B, int64_t M,
-                     int64_t N, int64_t K, void* Y, cudaStream_t stream) {
+                     const float* row_scale, const void* T, const void* W, const void* bias,
+                     const void* B, int64_t M, int64_t N, int64_t K, void* Y, cudaStream_t stream) {
   GemmLaunch p;
   std::memset(&p, 0, sizeof(p));
   const int bn = gemm_bn(N);
@@ -142,6 +168,7 @@ lynx_status run_gemm(DeviceState* ds, const void* a_src, bool sparse, const void
       return LYNX_ERR_CUDA;
   }
   p.meta = static_cast<const uint8_t*>(meta);
+  p.row_scale = row_scale;
   p.bias = bias;
   p.y = Y;
   p.M = M;
@@ -219,17 +246,28 @@ size_t lynx_workspace_bytes(int64_t M, int64_t N, int64_t K, int64_t r) {
   return workspace_layout(M, K, r).total;
 }
 
+size_t lynx_sparsify_workspace_bytes(int64_t M, int64_t K) {
+  if (M <= 0 || K <= 0) return 0;
+  return sparsify_workspace(M).total;
+}
+
 int lynx_sparsify(const void* X, int64_t M, int64_t K, void* vals, void* meta, float* row_scale,
-                  void* stream) {
-  if (X == nullptr || vals == nullptr || meta == nullptr) return LYNX_ERR_INVALID_ARG;
+                  void* workspace, size_t workspace_bytes, void* stream) {
+  if (X == nullptr || vals == nullptr || meta == nullptr || workspace == nullptr)
+    return LYNX_ERR_INVALID_ARG;
   lynx_status st = check_shape(M, 0, K);
   if (st != LYNX_OK) return st;
-  if (!aligned16(X) || !aligned16(vals) || !aligned16(meta) ||
+  if (!aligned16(X) || !aligned16(vals) || !aligned16(meta) || !aligned16(workspace) ||
       (reinterpret_cast<uintptr_t>(row_scale) & 3u) != 0)
     return LYNX_ERR_MISALIGNED;
+  const SparsifyWorkspace wl = sparsify_workspace(M);
+  if (workspace_bytes < wl.total) return LYNX_ERR_WORKSPACE_TOO_SMALL;
   DeviceState* ds = device_state();
   if (ds == nullptr) return LYNX_ERR_CUDA;
-  return run_sparsify(ds, X, nullptr, M, K, vals, meta, row_scale, nullptr, kModeSelect,
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  float* scale = row_scale ? row_scale : reinterpret_cast<float*>(ws + wl.scale);
+  return run_sparsify(ds, X, nullptr, M, K, vals, meta, scale, nullptr,
+                      reinterpret_cast<float2*>(ws + wl.lpart), nullptr, kModeSelect | kModeScaled,
                       static_cast<cudaStream_t>(stream));
 }
 
@@ -257,15 +295,22 @@ int lynx_linear(const void* X, const void* W, const void* bias, const void* A, c
   if (!skip_sparsify) {
     st = run_sparsify(ds, X, A, M, K, ws + wl.vals, ws + wl.meta,
                       reinterpret_cast<float*>(ws + wl.scale), t_buf,
+                      reinterpret_cast<float2*>(ws + wl.lpart), reinterpret_cast<float*>(ws + wl.tpart),
                       kModeSelect | (lora ? kModeLora : 0), s);
     if (st != LYNX_OK) return st;
-    return run_gemm(ds, ws + wl.vals, true, ws + wl.meta, t_buf, W, bias, B, M, N, K, Y, s);
+    if (void* ev = g_split_event.load())
+      if (cudaEventRecord(static_cast<cudaEvent_t>(ev), s) != cudaSuccess) return LYNX_ERR_CUDA;
+    return run_gemm(ds, ws + wl.vals, true, ws + wl.meta, reinterpret_cast<const float*>(ws + wl.scale),
+                    t_buf, W, bias, B, M, N, K, Y, s);
   }
   if (lora) {
-    st = run_sparsify(ds, X, A, M, K, nullptr, nullptr, nullptr, t_buf, kModeLora, s);
+    st = run_sparsify(ds, X, A, M, K, nullptr, nullptr, nullptr, t_buf, nullptr,
+                      reinterpret_cast<float*>(ws + wl.tpart), kModeLora, s);
     if (st != LYNX_OK) return st;
   }
-  return run_gemm(ds, X, false, nullptr, t_buf, W, bias, B, M, N, K, Y, s);
+  if (void* ev = g_split_event.load())
+    if (cudaEventRecord(static_cast<cudaEvent_t>(ev), s) != cudaSuccess) return LYNX_ERR_CUDA;
+  return run_gemm(ds, X, false, nullptr, nullptr, t_buf, W, bias, B, M, N, K, Y, s);
 }
 
 int lynx_linear_dense(const void* X, const void* W, const void* bias, const void* A,
@@ -287,7 +332,8 @@ int lynx_sparse_gemm(const void* vals, const void* meta, const void* T, const vo
     return LYNX_ERR_MISALIGNED;
   DeviceState* ds = device_state();
   if (ds == nullptr) return LYNX_ERR_CUDA;
-  return run_gemm(ds, vals, true, meta, T, W, bias, B, M, N, K, Y, static_cast<cudaStream_t>(stream));
+  return run_gemm(ds, vals, true, meta, nullptr, T, W, bias, B, M, N, K, Y,
+                  static_cast<cudaStream_t>(stream));
 }
 
 int lynx_check_error(void* stream, uint32_t* device_code) {
@@ -367,5 +413,7 @@ int lynx_meta_canonical_to_hw(const uint8_t* canonical, uint8_t* hw, int64_t M, 
 }
 
 int lynx_debug_set_stall(int enable) { return g_stall.exchange(enable ? 1 : 0); }
+
+void* lynx_profile_set_split_event(void* event) { return g_split_event.exchange(event); }
 
 }  // extern "C"

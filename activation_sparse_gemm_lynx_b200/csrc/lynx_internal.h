@@ -15,26 +15,36 @@ constexpr int kMetaBlockBytes = 2048;  // 128 TMEM lanes x 16 bytes
 
 // ---- sparsify / LoRA-down pass ---------------------------------------------
 
-enum SparsifyMode : int { kModeSelect = 1, kModeLora = 2 };
+// kModeSelect: S(X) (kept values + metadata + s); kModeLora: T = X A^T;
+// kModeScaled: values leave compensated (standalone S(X)), otherwise they
+// leave as kept and s is applied by the GEMM (T is then written as T / s).
+enum SparsifyMode : int { kModeSelect = 1, kModeLora = 2, kModeScaled = 4 };
+
+constexpr int kMaxSplit = 8;  // K ranges per row block in the sparsify pass
 
 struct SparsifyLaunch {
   CUtensorMap tm_x;     // X [M,K] bf16, box 64 x 128, 128B swizzle
   CUtensorMap tm_a;     // A [64,K] bf16, box 64 x 64, 128B swizzle (mode & kModeLora)
+  CUtensorMap tm_vals;  // vals [M,K/2] bf16, box 32 x 128, 64B swizzle (stores)
   void* vals;           // [M, K/2] bf16 (mode & kModeSelect)
   uint8_t* meta;        // hardware-layout metadata blocks (mode & kModeSelect)
-  float* row_scale;     // [M] or null
+  float* row_scale;     // [M] s per row (mode & kModeSelect)
   void* t_out;          // [M, 64] bf16 (mode & kModeLora)
+  float2* lpart;        // [split][M] partial (sum|x|, sum|kept|) per K range
+  float* tpart;         // [split][M][64] partial T per K range
   int64_t M, K;
   int mode;
-  int cluster;          // CTAs per row block along K (1, 2, 4 or 8)
+  int split;            // K ranges per row block (1..kMaxSplit, divides K/64)
   int boxes_per_cta;    // 64-column boxes each CTA covers
   int kblocks;          // metadata blocks per row block: ceil(K/128)
   int stall_test;       // test-only: the producer never loads, waits must time out
   uint32_t* status;     // device status word (first error code wins)
 };
 
+// sparsify pass + finalize (+ rescale for the standalone form), on one stream
 cudaError_t launch_sparsify(const SparsifyLaunch& p, cudaStream_t stream);
-int choose_sparsify_cluster(int64_t M, int64_t K, int num_sms);
+int choose_sparsify_split(int64_t M, int64_t K, int num_sms);
+size_t sparsify_smem_bytes();
 
 // ---- tcgen05 GEMM with LoRA-up + bias epilogue ------------------------------
 
@@ -45,6 +55,7 @@ struct GemmLaunch {
   CUtensorMap tm_lb;    // B [N,64] box 32 x BN, SW64 (lora)
   const uint8_t* meta;  // hardware metadata blocks (sparse)
   const void* bias;     // [N] bf16 or null
+  const float* row_scale;  // [M] fp32 multiplier of each accumulator row, or null
   void* y;              // [M,N] bf16
   int64_t M, N, K;
   int sparse;

@@ -5,34 +5,41 @@
 // ai-feeds.com summary "core module 1"):
 //   per token row m and group g of 4 consecutive K values: keep the 2 largest
 //   magnitudes (ties to the lower index); L_all = sum|x|, L_kept = sum|kept|
-//   (fp32); s = L_all / L_kept (1 if L_kept == 0); kept values v' = bf16(v*s),
-//   stored compressed (2 per group, ascending position) together with the
-//   2-bit positions in the operand layout of tcgen05.mma.sp; optionally
-//   T = X A^T (fp32 accumulate on tensor cores, stored as bf16).
+//   (fp32); s = L_all / L_kept (1 if L_kept == 0); the kept values, 2 per
+//   group in ascending position, and their 2-bit positions in the operand
+//   layout of tcgen05.mma.sp; optionally T = X A^T (fp32 accumulate on tensor
+//   cores).
 //
-// Organisation (one launch):
-//   grid = (C, ceil(M/128)), cluster = (C,1,1): the C CTAs of a cluster share
-//   one 128-row block and split K into C equal ranges.
+// Three kernels:
+//   sparsify_kernel  grid (C, ceil(M/128)): CTA (j, mb) covers rows
+//                    [128 mb, 128 mb + 128) and dense columns [j K/C, (j+1) K/C).
+//                    It writes the metadata and the kept values of its range
+//                    (as they are, exact copies of X) and fp32 partials: the two
+//                    row sums of its range and, with LoRA, T over its range.
+//   finalize_kernel  per row: combines the C partials in a fixed order
+//                    (deterministic) into s and T, written as bf16(T / s) when
+//                    the GEMM applies s to its accumulator row (so that
+//                    s * (S0 W^T + (T/s) B^T) = S(X) W^T + T B^T), else bf16(T).
+//   rescale_kernel   standalone S(X): kept values v -> bf16(v * s).
+//
+// sparsify_kernel, per CTA (2 CTAs per SM):
 //   warp 0      TMA producer: 128x64 tiles of X (and 64x64 tiles of A) into a
 //               3-stage ring (128-byte swizzle, the UMMA K-major layout)
-//   warp 1      owns TMEM (64 columns) and issues tcgen05.mma M=128,N=64,K=16
-//               on each X tile for the LoRA down-projection
-//   warps 2..9  256 "row threads": thread = (row, half of each 64-wide tile).
-//               Selection, fp32 partial sums, unscaled kept values and
-//               metadata go out as the tiles stream by.
-//   After the ring: partial sums of the C CTAs are combined in a fixed order
-//   over distributed shared memory (deterministic), every CTA derives s, the
-//   T partials are reduced column-slice-wise the same way, and a second sweep
-//   rescales the kept values this thread wrote moments ago (an L2 hit).
+//   warp 1      owns TMEM (64 columns), issues tcgen05.mma M=128,N=64,K=16 on
+//               each X tile for the LoRA down-projection
+//   warps 2-17  512 row threads: thread = (row, quarter of each 64-wide tile,
+//               i.e. 16 columns = 4 groups = one 16-bit metadata field); the
+//               kept values of a tile leave through one TMA store.
 //
-// Metadata layout (what tcgen05.cp.128x128b + tcgen05.mma.sp kind::f16 with
-// M=128 consume): one 2048-byte block per 128 rows x 128 dense K, stored as
-// 128 TMEM lanes x 16 bytes.  For row m (within the block) and dense column k
-// (within the block): lane = (m & 7) + 8*((k >> 4) & 1) + 16*(m >> 4), 32-bit
-// word = k >> 5, bit = (k & 15) + 16*((m >> 3) & 1) with 4 bits per group:
-// the group's nibble lo | hi << 2.  Blocks are ordered row-block major:
-// block (mb, kb) starts at byte (mb * ceil(K/128) + kb) * 2048.
+// Metadata layout (consumed by tcgen05.cp.128x128b + tcgen05.mma.sp kind::f16,
+// M=128): one 2048-byte block per 128 rows x 128 dense K, 128 TMEM lanes x 16
+// bytes.  Row m, dense column k (both within the block): lane = (m & 7) +
+// 8*((k >> 4) & 1) + 16*(m >> 4), 32-bit word k >> 5, bit (k & 15) +
+// 16*((m >> 3) & 1); 4 bits per group: lo | hi << 2.  Blocks are ordered row
+// block major: block (mb, kb) starts at byte (mb * ceil(K/128) + kb) * 2048.
 #include <cuda_bf16.h>
+
+#include <algorithm>
 
 #include "lynx_internal.h"
 #include "lynx_ptx.cuh"
@@ -42,37 +49,53 @@ namespace lynx {
 namespace {
 
 constexpr int kStages = 3;
-constexpr int kComputeWarps = 8;
-constexpr int kThreads = 64 + 32 * kComputeWarps;  // 320
-constexpr uint32_t kXTileBytes = 128 * 64 * 2;       // 16 KB
-constexpr uint32_t kATileBytes = 64 * 64 * 2;        // 8 KB
+constexpr int kComputeWarps = 16;
+constexpr int kComputeThreads = 32 * kComputeWarps;  // 512
+constexpr int kThreads = 64 + kComputeThreads;        // 576
+constexpr uint32_t kXTileBytes = 128 * 64 * 2;        // 16 KB
+constexpr uint32_t kATileBytes = 64 * 64 * 2;         // 8 KB
+constexpr uint32_t kStoreTileBytes = 128 * 32 * 2;    // 8 KB: 128 rows x 32 kept values
 constexpr uint32_t kTmemCols = 64;
+constexpr uint32_t kBarCompute = 1;                   // named barrier of the row threads
 
 struct __align__(1024) SparsifySmem {
   uint8_t xring[kStages][kXTileBytes];
   uint8_t aring[kStages][kATileBytes];
-  float recv[128 * 64];          // T partial slices from every CTA of the cluster
-  float2 part[128];              // this CTA's (L_all, L_kept) per row
-  float2 halfpart[128];          // second half-tile partials, combined locally
-  float srow[128];               // final s per row
+  uint8_t vstage[2][kStoreTileBytes];  // kept values of one tile, 64-byte swizzle
+  float2 quarter[3][128];              // partial sums of quarters 1..3
   uint64_t full[kStages];
-  uint64_t empty[kStages];
+  uint64_t empty[kStages];     // row threads done with a stage (one arrival per warp)
+  uint64_t mma_done[kStages];  // the LoRA MMAs done with a stage (tcgen05.commit)
   uint64_t tdone;
   uint64_t drain;
   uint32_t tmem_base;
   volatile uint32_t abort_flag;
 };
 
-__device__ __forceinline__ float abs_lo(uint32_t w) { return __uint_as_float((w << 16) & 0x7FFFFFFFu); }
-__device__ __forceinline__ float abs_hi(uint32_t w) { return __uint_as_float(w & 0x7FFF0000u); }
+__device__ __forceinline__ uint64_t pack_f2(float lo, float hi) {
+  return static_cast<uint64_t>(__float_as_uint(lo)) |
+         (static_cast<uint64_t>(__float_as_uint(hi)) << 32);
+}
+
+// (a.x + b.x, a.y + b.y), each an IEEE fp32 add rounded to nearest even
+__device__ __forceinline__ uint64_t add_f32x2(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+
+// |x| of both bf16 halves of w, widened to fp32 (exact): (low half, high half)
+__device__ __forceinline__ uint64_t abs_pair(uint32_t w) {
+  const uint32_t a = w & 0x7FFF7FFFu;
+  return pack_f2(__uint_as_float(a << 16), __uint_as_float(a & 0xFFFF0000u));
+}
 
 // Top-2 of the 4 bf16 values in (w0 = x1:x0, w1 = x3:x2) by magnitude, ties to
-// the lower index.  Each value becomes a distinct key (|x| << 2) | (3 - i), so
-// a larger key is a larger magnitude or, on equal magnitude, a lower index.
-// Returns the nibble lo | hi << 2 and the kept pair packed (x_lo in the low
-// half), and adds the group's magnitudes to the running fp32 sums in k order.
-__device__ __forceinline__ uint32_t select_group(uint32_t w0, uint32_t w1, uint32_t& kept,
-                                                 float& l_all, float& l_kept) {
+// the lower index.  Each value becomes a distinct key (|x| << 2) | (3 - i), so a
+// larger key is a larger magnitude or, on equal magnitude, a lower index; the
+// two largest keys come out of a 4-input max/min network.  Returns the nibble
+// lo | hi << 2 and the kept pair packed (x_lo in the low half).
+__device__ __forceinline__ uint32_t select_group(uint32_t w0, uint32_t w1, uint32_t& kept) {
   const uint32_t k0 = ((w0 << 2) & 0x1FFFCu) | 3u;
   const uint32_t k1 = ((w0 >> 14) & 0x1FFFCu) | 2u;
   const uint32_t k2 = ((w1 << 2) & 0x1FFFCu) | 1u;
@@ -85,14 +108,7 @@ __device__ __forceinline__ uint32_t select_group(uint32_t w0, uint32_t w1, uint3
   const uint32_t lo = 3u - max(a, b);
   const uint32_t hi = 3u - min(a, b);
   // byte selector picking elements lo and hi out of the 8 bytes (w1:w0)
-  const uint32_t sel = 0x1010u + lo * 0x22u + hi * 0x2200u;
-  kept = __byte_perm(w0, w1, sel);
-  l_all = __fadd_rn(l_all, abs_lo(w0));
-  l_all = __fadd_rn(l_all, abs_hi(w0));
-  l_all = __fadd_rn(l_all, abs_lo(w1));
-  l_all = __fadd_rn(l_all, abs_hi(w1));
-  l_kept = __fadd_rn(l_kept, abs_lo(kept));
-  l_kept = __fadd_rn(l_kept, abs_hi(kept));
+  kept = __byte_perm(w0, w1, 0x1010u + lo * 0x22u + hi * 0x2200u);
   return lo | (hi << 2);
 }
 
@@ -116,18 +132,18 @@ sparsify_kernel(const __grid_constant__ SparsifyLaunch p) {
 
   const uint32_t warp = warp_id_sync();
   const uint32_t lane = lane_id();
-  const uint32_t rank = cluster_ctarank();   // == blockIdx.x
-  const uint32_t C = static_cast<uint32_t>(p.cluster);
-  const int64_t mb = blockIdx.y;
+  const uint32_t j = blockIdx.x;  // K range
+  const int64_t mb = blockIdx.y;  // row block
   const int nboxes = p.boxes_per_cta;
   const bool do_sel = (p.mode & kModeSelect) != 0;
   const bool do_lora = (p.mode & kModeLora) != 0;
-  const int64_t kcol0 = static_cast<int64_t>(rank) * nboxes * 64;
+  const int64_t kcol0 = static_cast<int64_t>(j) * nboxes * 64;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&sm.full[s], 1);
-      mbar_init(&sm.empty[s], (do_sel ? kComputeWarps : 0) + (do_lora ? 1 : 0));
+      mbar_init(&sm.empty[s], kComputeWarps);
+      mbar_init(&sm.mma_done[s], 1);
     }
     mbar_init(&sm.tdone, 1);
     mbar_init(&sm.drain, 1);
@@ -154,7 +170,9 @@ sparsify_kernel(const __grid_constant__ SparsifyLaunch p) {
           const int slot = b % kStages;
           const uint32_t it = static_cast<uint32_t>(b / kStages);
           if (sm.abort_flag) break;
-          if (!mbar_wait(&sm.empty[slot], (it & 1u) ^ 1u)) {
+          // a stage is free once the row threads and the LoRA MMAs are done with it
+          if ((do_sel && !mbar_wait(&sm.empty[slot], (it & 1u) ^ 1u)) ||
+              (do_lora && !mbar_wait(&sm.mma_done[slot], (it & 1u) ^ 1u))) {
             set_abort(sm, p.status, kDevTimeoutEmpty);
             break;
           }
@@ -167,7 +185,8 @@ sparsify_kernel(const __grid_constant__ SparsifyLaunch p) {
       }
       // never leave with copies in flight: wait for the last fill of each slot
       for (int b = issued - 1; b >= 0 && b >= issued - kStages; --b) {
-        if (!mbar_wait(&sm.full[b % kStages], static_cast<uint32_t>(b / kStages) & 1u, kWaitLimitNs / 4))
+        if (!mbar_wait(&sm.full[b % kStages], static_cast<uint32_t>(b / kStages) & 1u,
+                       kWaitLimitNs / 4))
           record_error(p.status, kDevTimeoutDrain);
       }
     }
@@ -193,93 +212,112 @@ sparsify_kernel(const __grid_constant__ SparsifyLaunch p) {
           const uint64_t db = make_sdesc(aa + 32 * kk, 16, 1024, kSw128);
           mma_bf16(t_tmem, da, db, idesc, (b | kk) != 0 ? 1u : 0u);
         }
-        tc_commit(&sm.empty[slot]);
+        tc_commit(&sm.mma_done[slot]);
       }
       tc_commit(&sm.tdone);
-      // all MMAs issued so far are complete once this fires (used on every path)
+      // fires once every MMA issued above has completed (used on every path)
       tc_commit(&sm.drain);
       if (!mbar_wait(&sm.drain, 0)) record_error(p.status, kDevTimeoutDrain);
     }
     __syncwarp();
   } else if (do_sel) {
     // ------------------------------------------------------------ row threads
-    const uint32_t half = (warp - 2) >> 2;
+    const uint32_t ct = threadIdx.x - 64;     // 0..511
+    const uint32_t qt = (warp - 2) >> 2;      // which 16 columns of each tile
     const uint32_t row = 32 * (warp & 3) + lane;
     const int64_t grow = mb * 128 + row;
-    const bool row_ok = grow < p.M;
-    const uint32_t meta_lane0 = (row & 7) + 16 * (row >> 4);
+    // metadata: this thread's 16 columns form one 16-bit field of one lane
+    const uint32_t meta_lane = (row & 7) + 8 * (qt & 1) + 16 * (row >> 4);
     const uint32_t meta_hsel = (row >> 3) & 1;
-    uint16_t* meta_blk_base =
+    uint16_t* meta_row_blocks =
         reinterpret_cast<uint16_t*>(p.meta + static_cast<size_t>(mb) * p.kblocks * kMetaBlockBytes);
-    uint4* vrow = reinterpret_cast<uint4*>(static_cast<uint8_t*>(p.vals) +
-                                           static_cast<size_t>(grow) * p.K);  // K/2 bf16 = K bytes
-    float l_all = 0.f, l_kept = 0.f;
-    for (int b = 0; b < nboxes; ++b) {
+    // where this thread's 8 kept values sit in the 64-byte-swizzled store tile
+    const uint32_t vst_off = row * 64 + ((qt ^ ((row >> 1) & 3)) << 4);
+    uint64_t la2 = 0, lk2 = 0;  // (even, odd) fp32 partial sums
+    bool stop = false;
+    for (int b = 0; b < nboxes && !stop; ++b) {
       const int slot = b % kStages;
       const uint32_t it = static_cast<uint32_t>(b / kStages);
-      if (sm.abort_flag) break;
-      if (!mbar_wait(&sm.full[slot], it & 1u)) {
+      bool ok = !sm.abort_flag;
+      if (ok && !mbar_wait(&sm.full[slot], it & 1u)) {
         set_abort(sm, p.status, kDevTimeoutFull);
-        break;
+        ok = false;
       }
-      const uint8_t* tile = sm.xring[slot];
-      uint32_t kw[8];
-      uint32_t nib16[2];
+      ok = __all_sync(0xffffffffu, ok);
+      if (ok) {
+        const uint8_t* tile = sm.xring[slot];
+        uint32_t kw[4];
+        uint32_t nib = 0;
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const uint32_t chunk = 4 * half + q;
-        const uint4 v = *reinterpret_cast<const uint4*>(tile + row * 128 + ((chunk ^ (row & 7)) << 4));
-        const uint32_t n0 = select_group(v.x, v.y, kw[2 * q], l_all, l_kept);
-        const uint32_t n1 = select_group(v.z, v.w, kw[2 * q + 1], l_all, l_kept);
-        const uint32_t bits8 = n0 | (n1 << 4);
-        if (q & 1)
-          nib16[q >> 1] |= bits8 << 8;
-        else
-          nib16[q >> 1] = bits8;
+        for (int h = 0; h < 2; ++h) {
+          const uint32_t chunk = 2 * qt + h;
+          const uint4 v =
+              *reinterpret_cast<const uint4*>(tile + row * 128 + ((chunk ^ (row & 7)) << 4));
+          const uint32_t n0 = select_group(v.x, v.y, kw[2 * h]);
+          const uint32_t n1 = select_group(v.z, v.w, kw[2 * h + 1]);
+          nib |= (n0 | (n1 << 4)) << (8 * h);
+          la2 = add_f32x2(la2, abs_pair(v.x));
+          la2 = add_f32x2(la2, abs_pair(v.y));
+          la2 = add_f32x2(la2, abs_pair(v.z));
+          la2 = add_f32x2(la2, abs_pair(v.w));
+          lk2 = add_f32x2(lk2, abs_pair(kw[2 * h]));
+          lk2 = add_f32x2(lk2, abs_pair(kw[2 * h + 1]));
+        }
+        const int64_t kabs = kcol0 + 64 * b + 16 * qt;
+        uint16_t* blk = meta_row_blocks + static_cast<size_t>(kabs >> 7) * (kMetaBlockBytes / 2);
+        blk[meta_lane * 8 + static_cast<uint32_t>((kabs & 127) >> 5) * 2 + meta_hsel] =
+            static_cast<uint16_t>(nib);
+        *reinterpret_cast<uint4*>(sm.vstage[b & 1] + vst_off) = make_uint4(kw[0], kw[1], kw[2], kw[3]);
+        fence_proxy_async_smem();
+        // release the stage only after everything derived from it has been
+        // produced: an arrive does not wait for this warp's loads in flight
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.empty[slot]);
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&sm.empty[slot]);
-      // metadata: this thread covers dense columns [kabs, kabs+32) of its row
-      const int64_t kabs = kcol0 + 64 * b + 32 * half;
-      const int64_t kb = kabs >> 7;
-      const uint32_t c32 = static_cast<uint32_t>((kabs & 127) >> 5);
-      uint16_t* blk = meta_blk_base + static_cast<size_t>(kb) * (kMetaBlockBytes / 2);
-      blk[(meta_lane0) * 8 + c32 * 2 + meta_hsel] = static_cast<uint16_t>(nib16[0]);
-      blk[(meta_lane0 + 8) * 8 + c32 * 2 + meta_hsel] = static_cast<uint16_t>(nib16[1]);
-      if (row_ok) {
-        uint4* dst = vrow + (kabs >> 4);  // kabs/2 bf16 = kabs bytes = kabs/16 uint4
-        dst[0] = make_uint4(kw[0], kw[1], kw[2], kw[3]);
-        dst[1] = make_uint4(kw[4], kw[5], kw[6], kw[7]);
+      if (ct == 0) bulk_wait_read_all();  // the store of tile b-1 has read its buffer
+      stop = named_bar_red_or(kBarCompute, kComputeThreads, !ok);
+      if (!stop && ct == 0) {
+        tma_store_2d(&p.tm_vals, sm.vstage[b & 1], static_cast<int32_t>((kcol0 + 64 * b) / 2),
+                     static_cast<int32_t>(mb * 128));
+        bulk_commit();
       }
     }
-    if (half == 1) sm.halfpart[row] = make_float2(l_all, l_kept);
-    named_bar_sync(1, 32 * kComputeWarps);
-    if (half == 0) {
-      const float2 o = sm.halfpart[row];
-      sm.part[row] = make_float2(__fadd_rn(l_all, o.x), __fadd_rn(l_kept, o.y));
+    const float my_la = __fadd_rn(__uint_as_float(static_cast<uint32_t>(la2)),
+                                  __uint_as_float(static_cast<uint32_t>(la2 >> 32)));
+    const float my_lk = __fadd_rn(__uint_as_float(static_cast<uint32_t>(lk2)),
+                                  __uint_as_float(static_cast<uint32_t>(lk2 >> 32)));
+    if (qt > 0) sm.quarter[qt - 1][row] = make_float2(my_la, my_lk);
+    named_bar_sync(kBarCompute, kComputeThreads);
+    if (qt == 0 && grow < p.M) {
+      float a = my_la, k = my_lk;
+#pragma unroll
+      for (int q = 0; q < 3; ++q) {  // fixed order
+        const float2 o = sm.quarter[q][row];
+        a = __fadd_rn(a, o.x);
+        k = __fadd_rn(k, o.y);
+      }
+      p.lpart[static_cast<size_t>(j) * p.M + grow] = make_float2(a, k);
     }
+    if (ct == 0) bulk_wait_all();  // every value tile is in global memory
   }
 
-  // ---- T partial: TMEM -> registers -> owner CTA's receive buffer (by column slice)
+  // ---- T partial of this K range: TMEM -> registers -> global (fp32)
   if (do_lora && warp >= 2 && warp < 6) {
     const uint32_t row = 32 * (warp & 3) + lane;
+    const int64_t grow = mb * 128 + row;
     if (!sm.abort_flag && mbar_wait(&sm.tdone, 0)) {
       tc_fence_after();
-      const uint32_t w = kLoraRank / C;  // columns owned by each CTA
+      float4* dst = reinterpret_cast<float4*>(p.tpart + (static_cast<size_t>(j) * p.M + grow) * kLoraRank);
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         uint32_t r[32];
         tmem_ld_32x32b_x32(sm.tmem_base + ((32u * (warp & 3)) << 16) + 32u * h, r);
         tmem_ld_wait();
+        if (grow < p.M) {
 #pragma unroll
-        for (int c = 0; c < 32; c += 4) {
-          const uint32_t col = 32 * h + c;
-          const uint32_t owner = col / w;
-          const uint32_t off = col % w;
-          const uint32_t dst = mapa_shared(
-              smem_u32(&sm.recv[(rank * 128 + row) * w + off]), owner);
-          st_cluster_v4(dst, __uint_as_float(r[c]), __uint_as_float(r[c + 1]),
-                        __uint_as_float(r[c + 2]), __uint_as_float(r[c + 3]));
+          for (int c = 0; c < 32; c += 4)
+            dst[(32 * h + c) / 4] = make_float4(__uint_as_float(r[c]), __uint_as_float(r[c + 1]),
+                                                __uint_as_float(r[c + 2]), __uint_as_float(r[c + 3]));
         }
       }
       tc_fence_before();
@@ -288,73 +326,73 @@ sparsify_kernel(const __grid_constant__ SparsifyLaunch p) {
     }
   }
 
-  __syncwarp();
-  cluster_sync_all();  // partial sums and T slices are published cluster-wide
-
-  if (warp >= 2 && warp < 6) {
-    const uint32_t row = 32 * (warp & 3) + lane;
-    const int64_t grow = mb * 128 + row;
-    if (do_sel) {
-      float la = 0.f, lk = 0.f;
-      const uint32_t my = smem_u32(&sm.part[row]);
-      for (uint32_t j = 0; j < C; ++j) {  // fixed order: deterministic and identical in all CTAs
-        const float2 v = ld_cluster_f32x2(mapa_shared(my, j));
-        la = __fadd_rn(la, v.x);
-        lk = __fadd_rn(lk, v.y);
-      }
-      const float s = (lk == 0.f) ? 1.f : __fdiv_rn(la, lk);
-      sm.srow[row] = s;
-      if (p.row_scale != nullptr && rank == 0 && grow < p.M) p.row_scale[grow] = s;
-    }
-    if (do_lora && grow < p.M) {
-      const uint32_t w = kLoraRank / C;
-      __nv_bfloat16* trow = static_cast<__nv_bfloat16*>(p.t_out) + grow * kLoraRank + rank * w;
-      for (uint32_t c = 0; c < w; c += 2) {
-        float a0 = 0.f, a1 = 0.f;
-        for (uint32_t j = 0; j < C; ++j) {
-          a0 = __fadd_rn(a0, sm.recv[(j * 128 + row) * w + c]);
-          a1 = __fadd_rn(a1, sm.recv[(j * 128 + row) * w + c + 1]);
-        }
-        *reinterpret_cast<__nv_bfloat162*>(trow + c) = __floats2bfloat162_rn(a0, a1);
-      }
-    }
-  }
-
-  __syncwarp();
-  cluster_sync_all();  // no CTA leaves while a peer may still read its shared memory
-
+  __syncthreads();
   if (warp == 1 && do_lora) tmem_dealloc(sm.tmem_base, kTmemCols);
+}
 
-  // ---- second sweep: compensated values (re-read what this thread wrote)
-  if (do_sel && warp >= 2 && !sm.abort_flag) {
-    const uint32_t half = (warp - 2) >> 2;
-    const uint32_t row = 32 * (warp & 3) + lane;
-    const int64_t grow = mb * 128 + row;
-    if (grow < p.M) {
-      const float s = sm.srow[row];
-      uint4* vrow = reinterpret_cast<uint4*>(static_cast<uint8_t*>(p.vals) + static_cast<size_t>(grow) * p.K);
-      for (int b = 0; b < nboxes; ++b) {
-        const int64_t kabs = kcol0 + 64 * b + 32 * half;
-        uint4* d = vrow + (kabs >> 4);
-        uint4 v0 = d[0], v1 = d[1];
-        v0 = make_uint4(scale_pair(v0.x, s), scale_pair(v0.y, s), scale_pair(v0.z, s), scale_pair(v0.w, s));
-        v1 = make_uint4(scale_pair(v1.x, s), scale_pair(v1.y, s), scale_pair(v1.z, s), scale_pair(v1.w, s));
-        d[0] = v0;
-        d[1] = v1;
-      }
+// One warp per row: s from the C partial sums, T from the C partial products
+// (fixed order), T written as bf16(T / s) when `divide`.
+__global__ void __launch_bounds__(256)
+finalize_kernel(const float2* __restrict__ lpart, const float* __restrict__ tpart, int64_t M,
+                int C, int do_scale, int do_lora, int divide, float* __restrict__ row_scale,
+                __nv_bfloat16* __restrict__ t_out) {
+  const int64_t row = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+  const uint32_t lane = threadIdx.x & 31u;
+  if (row >= M) return;
+  float s = 1.f;
+  if (do_scale) {
+    float la = 0.f, lk = 0.f;
+    for (int j = 0; j < C; ++j) {
+      const float2 v = __ldcg(lpart + static_cast<size_t>(j) * M + row);
+      la = __fadd_rn(la, v.x);
+      lk = __fadd_rn(lk, v.y);
     }
+    s = (lk == 0.f) ? 1.f : __fdiv_rn(la, lk);
+    if (lane == 0) row_scale[row] = s;
+  }
+  if (do_lora) {
+    float a0 = 0.f, a1 = 0.f;  // columns 2*lane, 2*lane+1
+    for (int j = 0; j < C; ++j) {
+      const float2 v = __ldcg(reinterpret_cast<const float2*>(
+          tpart + (static_cast<size_t>(j) * M + row) * kLoraRank) + lane);
+      a0 = __fadd_rn(a0, v.x);
+      a1 = __fadd_rn(a1, v.y);
+    }
+    if (divide) {
+      a0 = __fdiv_rn(a0, s);
+      a1 = __fdiv_rn(a1, s);
+    }
+    reinterpret_cast<__nv_bfloat162*>(t_out + row * kLoraRank)[lane] = __floats2bfloat162_rn(a0, a1);
+  }
+}
+
+// Standalone S(X): the kept values become bf16(v * s) in place.  One thread per
+// 8 values (16 bytes); rows of K/2 values.
+__global__ void __launch_bounds__(256)
+rescale_kernel(uint4* __restrict__ vals, const float* __restrict__ row_scale, int64_t M,
+               int64_t K) {
+  const int64_t per_row = K / 16;  // uint4 per row (K/2 bf16 = K bytes)
+  const int64_t total = M * per_row;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const float s = __ldg(row_scale + i / per_row);
+    const uint4 v = vals[i];
+    vals[i] = make_uint4(scale_pair(v.x, s), scale_pair(v.y, s), scale_pair(v.z, s), scale_pair(v.w, s));
   }
 }
 
 }  // namespace
 
-int choose_sparsify_cluster(int64_t M, int64_t K, int num_sms) {
+size_t sparsify_smem_bytes() { return sizeof(SparsifySmem) + 1024; }
+
+// K ranges per row block: the largest C <= kMaxSplit dividing the 64-column
+// boxes of a row such that C * ceil(M/128) CTAs fit in one wave (2 per SM).
+int choose_sparsify_split(int64_t M, int64_t K, int num_sms) {
   const int64_t row_blocks = (M + 127) / 128;
-  if (K % kMetaBlockK != 0) return 1;
-  const int64_t kblocks = K / kMetaBlockK;
+  const int64_t boxes = K / 64;
   int best = 1;
-  for (int c = 2; c <= 8; c *= 2) {
-    if (kblocks % c != 0) break;
+  for (int c = 2; c <= kMaxSplit; ++c) {
+    if (boxes % c != 0) continue;
     if (row_blocks * c > 2LL * num_sms) break;
     best = c;
   }
@@ -362,27 +400,34 @@ int choose_sparsify_cluster(int64_t M, int64_t K, int num_sms) {
 }
 
 cudaError_t launch_sparsify(const SparsifyLaunch& p, cudaStream_t stream) {
-  const size_t smem = sizeof(SparsifySmem) + 1024;
-  static bool configured = false;
-  if (!configured) {
+  const size_t smem = sparsify_smem_bytes();
+  static int configured_device = -1;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (configured_device != dev) {
     cudaError_t e = cudaFuncSetAttribute(sparsify_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
     if (e != cudaSuccess) return e;
-    configured = true;
+    configured_device = dev;
   }
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(p.cluster), static_cast<unsigned>((p.M + 127) / 128), 1);
-  cfg.blockDim = dim3(kThreads, 1, 1);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = static_cast<unsigned>(p.cluster);
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, sparsify_kernel, p);
+  const dim3 grid(static_cast<unsigned>(p.split), static_cast<unsigned>((p.M + 127) / 128), 1);
+  sparsify_kernel<<<grid, kThreads, smem, stream>>>(p);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const bool do_sel = (p.mode & kModeSelect) != 0;
+  const bool do_lora = (p.mode & kModeLora) != 0;
+  const bool scaled = (p.mode & kModeScaled) != 0;
+  const unsigned fin_blocks = static_cast<unsigned>((p.M + 7) / 8);
+  finalize_kernel<<<fin_blocks, 256, 0, stream>>>(p.lpart, p.tpart, p.M, p.split, do_sel ? 1 : 0,
+                                                  do_lora ? 1 : 0, (do_sel && !scaled) ? 1 : 0,
+                                                  p.row_scale,
+                                                  static_cast<__nv_bfloat16*>(p.t_out));
+  e = cudaGetLastError();
+  if (e != cudaSuccess || !(do_sel && scaled)) return e;
+  const int64_t n16 = p.M * (p.K / 16);
+  const unsigned rb = static_cast<unsigned>(std::min<int64_t>((n16 + 255) / 256, 4096));
+  rescale_kernel<<<rb, 256, 0, stream>>>(static_cast<uint4*>(p.vals), p.row_scale, p.M, p.K);
+  return cudaGetLastError();
 }
 
 }  // namespace lynx

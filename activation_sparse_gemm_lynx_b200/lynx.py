@@ -51,7 +51,8 @@ def library():
             "lynx_vals_bytes": ([i64, i64], sz),
             "lynx_meta_bytes": ([i64, i64], sz),
             "lynx_workspace_bytes": ([i64, i64, i64, i64], sz),
-            "lynx_sparsify": ([p, i64, i64, p, p, p, p], i32),
+            "lynx_sparsify_workspace_bytes": ([i64, i64], sz),
+            "lynx_sparsify": ([p, i64, i64, p, p, p, p, sz, p], i32),
             "lynx_linear": ([p, p, p, p, p, i64, i64, i64, i64, i32, p, p, sz, p], i32),
             "lynx_linear_dense": ([p, p, p, p, p, i64, i64, i64, i64, p, p, sz, p], i32),
             "lynx_sparse_gemm": ([p, p, p, p, p, p, i64, i64, i64, i64, p, p], i32),
@@ -59,6 +60,7 @@ def library():
             "lynx_meta_hw_to_canonical": ([p, p, i64, i64], i32),
             "lynx_meta_canonical_to_hw": ([p, p, i64, i64], i32),
             "lynx_debug_set_stall": ([i32], i32),
+            "lynx_profile_set_split_event": ([p], p),
         }
         for name, (args, res) in sigs.items():
             f = getattr(lib, name)
@@ -132,7 +134,12 @@ def _need(t, name, dtype=None, shape=None):
     return t
 
 
-def lynx_sparsify(X, vals=None, meta=None, row_scale=None, stream=None, want_scale=True):
+def lynx_sparsify_workspace_bytes(M, K):
+    return library().lynx_sparsify_workspace_bytes(M, K)
+
+
+def lynx_sparsify(X, vals=None, meta=None, row_scale=None, workspace=None, stream=None,
+                  want_scale=True):
     """S(X): returns (vals [M,K/2] bf16, meta uint8 [lynx_meta_bytes], row_scale [M] f32 or None)."""
     import torch
 
@@ -144,14 +151,18 @@ def lynx_sparsify(X, vals=None, meta=None, row_scale=None, stream=None, want_sca
         meta = torch.empty(lynx_meta_bytes(M, K), dtype=torch.uint8, device=X.device)
     if row_scale is None and want_scale:
         row_scale = torch.empty(M, dtype=torch.float32, device=X.device)
+    if workspace is None:
+        workspace = torch.empty(lynx_sparsify_workspace_bytes(M, K), dtype=torch.uint8,
+                                device=X.device)
     _need(vals, "vals", torch.bfloat16, (M, K // 2))
     _need(meta, "meta", torch.uint8)
+    _need(workspace, "workspace", torch.uint8)
     if meta.numel() < lynx_meta_bytes(M, K):
         raise ValueError("meta buffer too small")
     if row_scale is not None:
         _need(row_scale, "row_scale", torch.float32, (M,))
     st = library().lynx_sparsify(_ptr(X), M, K, _ptr(vals), _ptr(meta), _ptr(row_scale),
-                                 _stream(stream))
+                                 _ptr(workspace), workspace.numel(), _stream(stream))
     _check(st, "lynx_sparsify")
     return vals, meta, row_scale
 
@@ -279,6 +290,13 @@ def lynx_meta_canonical_to_hw(canonical, M, K):
                                              out.ctypes.data_as(ctypes.c_void_p), M, K)
     _check(st, "lynx_meta_canonical_to_hw")
     return out
+
+
+def lynx_profile_set_split_event(event):
+    """Record `event` (a torch.cuda.Event, or None) between the two kernels of
+    every later lynx_linear call (see include/lynx.h)."""
+    handle = None if event is None else ctypes.c_void_p(event.cuda_event)
+    return library().lynx_profile_set_split_event(handle)
 
 
 def lynx_debug_set_stall(enable):

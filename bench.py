@@ -1,0 +1,449 @@
+#!/usr/bin/env python
+"""Benchmark of the B200 RT-Lynx online 2:4 activation-sparse linear layer.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+    python bench.py --impl reference ...      # the CPU oracle, timed as it stands
+
+One step = one ``lynx_linear`` call (sparsify + LoRA-down pass, sparse GEMM with
+LoRA-up and bias epilogue) on one batch of the workload, inputs resident in
+HBM.  L2 is flushed (256 MiB write) before every step, outside the timed step;
+each step is timed with CUDA events on the launching stream.  The metric is the
+dense-equivalent throughput 2*M*N*K / t.  Alongside: a dense bf16 GEMM of the
+same shape (torch.matmul / cuBLAS, comparison only), this library's dense path,
+the per-kernel split (sparsify pass vs GEMM), an end-to-end number through the
+same call with pinned host buffers, clocks sampled during the timed region,
+the roofline of the dominant kernel and the CPU oracle's throughput on a
+bounded sample.
+
+Multi-GPU (torchrun, one process per GPU): token rows are independent, so each
+rank runs its own batch of the workload (weak scaling, no data-path
+collective); the step time is the maximum over ranks.
+"""
+import argparse
+import datetime
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "sparse-act linear dense-equiv TFLOP/s (2MNK/t) & speedup vs dense bf16 GEMM"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+# DRAM bytes (read + write) per launch of the sparse GEMM kernel from one ncu
+# capture of the same kernel, per workload; None until captured for the kernel
+# as it stands (see profiles/).
+GEMM_DRAM_TRAFFIC = {}
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["lynx", "reference"], default="lynx")
+    ap.add_argument("--workload", default="mlp_up")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0,
+                    help="approximate CPU time of the oracle baseline sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--only-linear", action="store_true",
+                    help="time the layer only (no comparisons, e2e or CPU baseline); "
+                         "the short launch sequence used for ncu captures")
+    return ap.parse_args(argv)
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": float(p["hbm_gbs"]), "bf16_tflops": float(p["bf16_tflops"]),
+                "bf16_tflops_sustained": float(p.get("bf16_tflops_sustained", p["bf16_tflops"])),
+                "source": "measured"}
+    except (OSError, KeyError, ValueError):
+        return dict(FALLBACK_PEAKS, source="fallback")
+
+
+def dist_env():
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("LOCAL_RANK", "0")),
+            int(os.environ.get("WORLD_SIZE", "1")))
+
+
+def max_over_ranks(value, world):
+    """Max of a float over all ranks (a timing reduction, not part of the layer)."""
+    if world == 1:
+        return value
+    import torch
+    import torch.distributed as dist
+
+    dev = torch.device("cuda", torch.cuda.current_device()) if dist.get_backend() == "nccl" \
+        else torch.device("cpu")
+    t = torch.tensor([value], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+
+
+def rank_seed(base_seed, rank):
+    """Each rank draws its own batch of the workload (same shapes)."""
+    return base_seed if rank == 0 else [base_seed, rank]
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region (NVML reads only; no setting is changed)
+
+class ClockSampler:
+    REASONS = {
+        0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+        0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown", 0x2: "applications_clocks_setting",
+    }
+
+    def __init__(self, torch_device_index):
+        self.samples = []
+        self.reasons = 0
+        self._stop = threading.Event()
+        self._thread = None
+        self.max_mhz = None
+        self.ok = False
+        try:
+            import pynvml
+
+            pynvml.nvmlInit()
+            import torch
+
+            uuid = str(torch.cuda.get_device_properties(torch_device_index).uuid)
+            h = None
+            for i in range(pynvml.nvmlDeviceGetCount()):
+                hh = pynvml.nvmlDeviceGetHandleByIndex(i)
+                u = pynvml.nvmlDeviceGetUUID(hh)
+                u = u.decode() if isinstance(u, bytes) else u
+                if u.replace("GPU-", "") == uuid.replace("GPU-", ""):
+                    h = hh
+            if h is None:
+                h = pynvml.nvmlDeviceGetHandleByIndex(torch_device_index)
+            self.h = h
+            self.nv = pynvml
+            self.max_mhz = float(pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM))
+            self.ok = True
+        except Exception as e:  # noqa: BLE001 - clocks are informative only
+            self.err = repr(e)
+
+    def _run(self):
+        nv = self.nv
+        get_reasons = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            getattr(nv, "nvmlDeviceGetCurrentClocksThrottleReasons")
+        while not self._stop.is_set():
+            try:
+                mhz = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
+                util = nv.nvmlDeviceGetUtilizationRates(self.h).gpu
+                r = get_reasons(self.h)
+                self.samples.append((float(mhz), int(util), int(r)))
+            except Exception:  # noqa: BLE001
+                pass
+            self._stop.wait(0.01)
+
+    def start(self):
+        if self.ok:
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+
+    def stop(self):
+        if self._thread is not None:
+            self._stop.set()
+            self._thread.join()
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0,
+                    "note": "NVML unavailable: " + getattr(self, "err", "")}
+        busy = [s for s in self.samples if s[1] > 0] or self.samples
+        reasons = 0
+        for s in busy:
+            reasons |= s[2]
+        names = sorted(n for bit, n in self.REASONS.items() if reasons & bit)
+        return {"sm_mhz": statistics.median(s[0] for s in busy) if busy else None,
+                "sm_max_mhz": self.max_mhz, "reasons": names, "samples": len(busy)}
+
+
+# ---------------------------------------------------------------------------
+# the CPU oracle on a bounded sample of the workload
+
+def oracle_sample(inp, rows, skip=False):
+    import oracle
+
+    X = inp["X"][:rows]
+    t0 = time.perf_counter()
+    oracle.linear(X, inp["W"], inp["bias"], inp["A"], inp["B"], skip=skip)
+    return time.perf_counter() - t0
+
+
+def calibrate_oracle_rows(inp, target_s, M):
+    import oracle
+
+    cores = oracle.num_threads()
+    rows = max(1, cores)
+    t = oracle_sample(inp, rows)
+    while t < target_s / 4 and rows < M:
+        rows = min(M, int(rows * max(2.0, target_s / max(t, 1e-3) / 2)))
+        t = oracle_sample(inp, rows)
+    rows = min(M, max(1, int(rows * target_s / max(t, 1e-3))))
+    return rows, cores
+
+
+def cpu_baseline(inp, shape, target_s):
+    rows, cores = calibrate_oracle_rows(inp, target_s, shape.M)
+    t = oracle_sample(inp, rows)
+    flops = 2.0 * rows * shape.N * shape.K
+    return {"value": flops / t / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+            "sample": f"{rows} of {shape.M} token rows of {shape.name} (rows are independent), "
+                      f"full N={shape.N} and K={shape.K}, fp64 C oracle, {t:.1f} s"}
+
+
+# ---------------------------------------------------------------------------
+
+
+def workload_desc(shape):
+    kind = "GELU(tanh) inputs" if shape.x_kind == "gelu" else "8% N(0,1) / 92% N(0,0.05) mixture"
+    return (f"{shape.name}: X[{shape.M},{shape.K}] -> Y[{shape.M},{shape.N}], LoRA r={shape.r}, "
+            f"bias, {kind}")
+
+
+def run_reference(args):
+    rank, _, world = dist_env()
+    if rank != 0:
+        return 0
+    from activation_sparse_gemm_lynx_b200 import workloads
+    import oracle
+
+    shape = workloads.CONFIGS[args.workload]
+    inp = workloads.make_config_inputs(args.workload)
+    per_step = max(1.0, min(8.0, 150.0 / max(1, args.steps + args.warmup)))
+    rows, cores = calibrate_oracle_rows(inp, per_step, shape.M)
+    for _ in range(args.warmup):
+        oracle_sample(inp, rows)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle_sample(inp, rows)
+    t = (time.perf_counter() - t0) / max(1, args.steps)
+    value = 2.0 * rows * shape.N * shape.K / t / 1e12
+    sample = (f"each step: {rows} of {shape.M} token rows of {shape.name} (rows are independent), "
+              f"full N and K, fp64 C oracle on {cores} threads")
+    out = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": t * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded)",
+        "config": {"workload": workload_desc(shape), "M": shape.M, "N": shape.N, "K": shape.K,
+                   "r": shape.r, "rows_per_step": rows},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+    print(json.dumps(out), flush=True)
+    return 0
+
+
+def run_lynx(args):
+    import numpy as np
+    import torch
+
+    from activation_sparse_gemm_lynx_b200 import lynx, workloads
+
+    rank, local_rank, world = dist_env()
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    torch.cuda.set_device(local_rank)
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    lynx.library()
+
+    shape = workloads.CONFIGS[args.workload]
+    M, N, K, r = shape.M, shape.N, shape.K, shape.r
+    inp = workloads.make_linear_inputs(M, K, N, r, seed=rank_seed(shape.seed, rank),
+                                       x_kind=shape.x_kind)
+
+    def dev(a):
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).cuda()
+
+    X, W, bias, A, B = (dev(inp[k]) for k in ("X", "W", "bias", "A", "B"))
+    Y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    Yd = torch.empty_like(Y)
+    ws = torch.empty(lynx.lynx_workspace_bytes(M, N, K, r), dtype=torch.uint8, device="cuda")
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.int32, device="cuda")
+    Xh = torch.from_numpy(inp["X"].view(np.int16)).view(torch.bfloat16).pin_memory()
+    Yh = torch.empty((M, N), dtype=torch.bfloat16).pin_memory()
+    Xe = torch.empty_like(X)
+
+    def step_linear():
+        lynx.lynx_linear(X, W, bias, A, B, Y=Y, workspace=ws)
+
+    def step_dense_lynx():
+        lynx.lynx_linear(X, W, bias, A, B, skip_sparsify=True, Y=Y, workspace=ws)
+
+    def step_dense_torch():
+        torch.matmul(X, W.t(), out=Yd)
+
+    def step_e2e():
+        Xe.copy_(Xh, non_blocking=True)
+        lynx.lynx_linear(Xe, W, bias, A, B, Y=Y, workspace=ws)
+        Yh.copy_(Y, non_blocking=True)
+
+    def timed(step, n, split=False):
+        """Per-step device times (ms) of n steps, L2 flushed before each."""
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(n)]
+        for trio in ev:        # create the CUDA events up front
+            for e in trio:
+                e.record()
+        torch.cuda.synchronize()
+        for i in range(n):
+            flush.zero_()
+            if split:
+                lynx.lynx_profile_set_split_event(ev[i][1])
+            ev[i][0].record()
+            step()
+            ev[i][2].record()
+        if split:
+            lynx.lynx_profile_set_split_event(None)
+        torch.cuda.synchronize()
+        tot = [ev[i][0].elapsed_time(ev[i][2]) for i in range(n)]
+        if split:
+            first = [ev[i][0].elapsed_time(ev[i][1]) for i in range(n)]
+            second = [ev[i][1].elapsed_time(ev[i][2]) for i in range(n)]
+            return tot, first, second
+        return tot
+
+    # warm-up (untimed)
+    for _ in range(args.warmup):
+        step_linear()
+    torch.cuda.synchronize()
+    st, code = lynx.lynx_check_error()
+    if st != lynx.LYNX_OK:
+        raise RuntimeError(f"device status after warm-up: {st} code {code:#x}")
+
+    clocks = ClockSampler(local_rank)
+    barrier(world)
+    torch.cuda.synchronize()
+    clocks.start()
+    tot, t_sp, t_gemm = timed(step_linear, args.steps, split=True)
+    torch.cuda.synchronize()
+    clock_info = clocks.stop()
+    barrier(world)
+    st, code = lynx.lynx_check_error()
+    if st != lynx.LYNX_OK:
+        raise RuntimeError(f"device status after timing: {st} code {code:#x}")
+
+    total_ms = max_over_ranks(sum(tot), world)
+    ms_step = total_ms / args.steps
+    sp_ms = statistics.mean(t_sp)
+    gemm_ms = statistics.mean(t_gemm)
+
+    if args.only_linear:
+        if world > 1:
+            import torch.distributed as dist
+
+            dist.destroy_process_group()
+        if rank == 0:
+            print(json.dumps({"metric": METRIC, "ms_per_step": ms_step, "sparsify_ms": sp_ms,
+                              "gemm_ms": gemm_ms, "n_gpus": world, "steps": args.steps,
+                              "warmup": args.warmup, "only_linear": True}), flush=True)
+        return 0
+
+    # comparisons (same process, same loop structure)
+    ncmp = max(3, min(args.steps, 50))
+    for _ in range(3):
+        step_dense_torch()
+    dense_ms = max_over_ranks(statistics.mean(timed(step_dense_torch, ncmp)), world)
+    for _ in range(3):
+        step_dense_lynx()
+    lynx_dense_ms = max_over_ranks(statistics.mean(timed(step_dense_lynx, ncmp)), world)
+    for _ in range(3):
+        step_e2e()
+    e2e_ms = max_over_ranks(statistics.mean(timed(step_e2e, ncmp)), world)
+
+    flops = 2.0 * M * N * K
+    peaks = load_peaks()
+    sparse_peak = 2.0 * peaks["bf16_tflops"]
+    gemm_tflops = flops / (gemm_ms * 1e-3) / 1e12
+    sp_bytes = 2 * M * K + M * K + lynx.lynx_meta_bytes(M, K) + 2 * M * r + 4 * M + 2 * r * K
+    sp_gbs = sp_bytes / (sp_ms * 1e-3) / 1e9
+    traffic = GEMM_DRAM_TRAFFIC.get(args.workload)
+
+    result = {
+        "metric": METRIC,
+        "value": world * flops / (ms_step * 1e-3) / 1e12,
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms_step,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded numpy draws rounded to bf16; random weights)",
+        "config": {
+            "workload": workload_desc(shape), "M": M, "N": N, "K": K, "r": r,
+            "l2": "flushed before every step (256 MiB write, outside the timed step)",
+            "parallelism": f"dp{world} (independent token-row batches per GPU, no collective)",
+        },
+        "speedup_vs_dense_bf16": dense_ms / ms_step,
+        "sparsify_overhead": sp_ms / ms_step,
+        "breakdown_ms": {"linear": ms_step, "sparsify_pass": sp_ms, "sparse_gemm": gemm_ms,
+                         "dense_torch_matmul": dense_ms, "lynx_dense_path": lynx_dense_ms},
+        "roofline": {
+            "bound": "tensor", "kernel": "lynx_gemm_kernel<256,sparse>",
+            "achieved": gemm_tflops, "peak": sparse_peak, "unit": "TFLOP/s",
+            "frac": gemm_tflops / sparse_peak, "traffic": traffic,
+            "peak_note": f"2 x {peaks['source']} dense bf16 burst ({peaks['bf16_tflops']} TFLOP/s); "
+                         "2:4 sparse runs at twice the dense rate",
+            "work": "2*M*N*K dense-equivalent flops per launch",
+        },
+        "roofline_sparsify": {
+            "bound": "hbm", "kernel": "sparsify_kernel", "achieved": sp_gbs,
+            "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": sp_gbs / peaks["hbm_gbs"],
+            "traffic": None,
+            "work": "X read 2MK + vals MK + meta MK/8 + T 2Mr + s 4M + A 2rK bytes",
+        },
+        "e2e": {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                "h2d_bytes_per_step": 2 * M * K, "d2h_bytes_per_step": 2 * M * N,
+                "ms_per_step": e2e_ms,
+                "note": "X copied from pinned host memory and Y copied back inside each step; "
+                        "weights resident"},
+        "gpu_launches": 2 * args.steps,
+        "clocks": clock_info,
+    }
+
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        result["cpu_baseline"] = cpu_baseline(inp, shape, args.cpu_seconds)
+
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+    return 0
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_lynx(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -90,11 +90,15 @@ LYNX_API size_t lynx_vals_bytes(int64_t M, int64_t K);
  * each group of 4 owns 4 bits: lo | hi << 2 (lo < hi its kept positions). */
 LYNX_API size_t lynx_meta_bytes(int64_t M, int64_t K);
 
-/* Bytes of the workspace lynx_linear needs (compressed values, metadata, row
- * scales, the bf16 LoRA down-projection T [M,64], alignment padding). */
+/* Bytes of the workspace lynx_linear needs (kept values, metadata, row scales,
+ * the bf16 LoRA down-projection [M,64], per-range partial sums, alignment). */
 LYNX_API size_t lynx_workspace_bytes(int64_t M, int64_t N, int64_t K, int64_t r);
 
 /* ---- the layer --------------------------------------------------------- */
+
+/* Bytes of the scratch workspace lynx_sparsify needs (per-range partial row
+ * sums and, when no row_scale buffer is given, s). */
+LYNX_API size_t lynx_sparsify_workspace_bytes(int64_t M, int64_t K);
 
 /* S(X) alone (qingkeai.online article sections 02-03.1; ai-feeds summary,
  * core module 1).
@@ -104,17 +108,23 @@ LYNX_API size_t lynx_workspace_bytes(int64_t M, int64_t N, int64_t K, int64_t r)
  *   meta      out: metadata blocks, lynx_meta_bytes(M,K) bytes (layout above);
  *             rows M..ceil(M/128)*128-1 hold the pattern of an all-zero row
  *   row_scale [M] fp32, out: s per row, or NULL
- * The vals buffer is also used as the pass's own scratch while it runs. */
-LYNX_API int lynx_sparsify(const void* X, int64_t M, int64_t K, void* vals, void* meta, float* row_scale,
-                  void* stream);
+ *   workspace caller-allocated scratch of workspace_bytes >=
+ *             lynx_sparsify_workspace_bytes(M,K) */
+LYNX_API int lynx_sparsify(const void* X, int64_t M, int64_t K, void* vals, void* meta,
+                           float* row_scale, void* workspace, size_t workspace_bytes,
+                           void* stream);
 
 /* Y = S(X) W^T + bias + (X A^T) B^T  (S(X) = X when skip_sparsify != 0).
  *   X [M,K], W [N,K] (frozen backbone weight), bias [N] or NULL,
  *   A [r,K] and B [N,r] (LoRA, both or neither; r must be 64), Y [M,N] out.
  *   workspace: caller-allocated device buffer of workspace_bytes >=
- *   lynx_workspace_bytes(M,N,K,r); after the call it holds S(X) (vals, meta,
- *   row scales) and T = X A^T as bf16, in that order at 256-byte aligned
- *   offsets.  Y is bf16(acc + bias) with acc accumulated in fp32. */
+ *   lynx_workspace_bytes(M,N,K,r), used as scratch; at 256-byte aligned
+ *   offsets, in this order, it ends up holding the kept values before
+ *   compensation [M,K/2] bf16, the metadata, s per row [M] fp32 and T/s [M,r]
+ *   bf16 (T = X A^T).
+ *   The compensation factor s is applied to the fp32 accumulator row, so
+ *   Y = bf16(s * (S0 W^T + (T/s) B^T) + bias) with S0 the uncompensated kept
+ *   values: the same product as S(X) W^T + T B^T with one rounding fewer. */
 LYNX_API int lynx_linear(const void* X, const void* W, const void* bias, const void* A, const void* B,
                 int64_t M, int64_t N, int64_t K, int64_t r, int skip_sparsify, void* Y,
                 void* workspace, size_t workspace_bytes, void* stream);
@@ -149,6 +159,13 @@ LYNX_API int lynx_check_error(void* stream, uint32_t* device_code);
  * and padding K with zero bits. */
 LYNX_API int lynx_meta_hw_to_canonical(const uint8_t* hw, uint8_t* canonical, int64_t M, int64_t K);
 LYNX_API int lynx_meta_canonical_to_hw(const uint8_t* canonical, uint8_t* hw, int64_t M, int64_t K);
+
+/* Profiling hook: when `event` (a cudaEvent_t passed as void*) is non-NULL,
+ * lynx_linear records it on its stream between the sparsify pass and the GEMM,
+ * so a caller can time the two kernels of one call separately with events
+ * recorded before and after the call.  NULL (the default) turns it off.
+ * Process-wide; returns the previous event. */
+LYNX_API void* lynx_profile_set_split_event(void* event);
 
 /* Test hook (not for production use): when nonzero, kernels launched after
  * this call never load their inputs, so their bounded waits run out (about 2 s)

@@ -83,3 +83,38 @@ def y_tolerance_check(y_gpu, y_ref, sx_rows, w_rows):
     worst = float((err / np.maximum(bound, 1e-30)).max())
     fro = float(np.linalg.norm(y_gpu - y_ref) / max(np.linalg.norm(y_ref), 1e-30))
     return worst, fro
+
+
+def kept_from_x(x_bits, canon, K):
+    """The uncompensated kept values (bf16 bits, [M, K/2]) at the positions the
+    canonical metadata names."""
+    M = x_bits.shape[0]
+    nib = np.empty((M, K // 4), dtype=np.uint8)
+    nib[:, 0::2] = canon & 0xF
+    nib[:, 1::2] = canon >> 4
+    lo = (nib & 3).astype(np.int64)
+    hi = ((nib >> 2) & 3).astype(np.int64)
+    g = np.asarray(x_bits, dtype=np.uint16).reshape(M, K // 4, 4)
+    rows = np.arange(M)[:, None]
+    grp = np.arange(K // 4)[None, :]
+    out = np.empty((M, K // 4, 2), dtype=np.uint16)
+    out[:, :, 0] = g[rows, grp, lo]
+    out[:, :, 1] = g[rows, grp, hi]
+    return out.reshape(M, K // 2)
+
+
+def workspace_views(raw, M, K, r=64):
+    """Split a lynx_linear workspace (numpy uint8) into its documented parts:
+    kept values [M,K/2] (bf16 bits), metadata bytes, s [M] f32, T/s [M,r] bf16 bits."""
+    def a256(x):
+        return (x + 255) // 256 * 256
+    kblocks = (K + 127) // 128
+    meta_bytes = (M + 127) // 128 * kblocks * 2048
+    o_meta = a256(M * K)
+    o_scale = a256(o_meta + meta_bytes)
+    o_t = a256(o_scale + 4 * M)
+    vals = raw[: M * K].view(np.uint16).reshape(M, K // 2)
+    meta = raw[o_meta: o_meta + meta_bytes]
+    scale = raw[o_scale: o_scale + 4 * M].view(np.float32)
+    t = raw[o_t: o_t + 2 * M * r].view(np.uint16).reshape(M, r)
+    return vals, meta, scale, t

@@ -81,10 +81,18 @@ def test_linear_argument_errors(lib):
 
 def test_sparsify_argument_errors(lib):
     f = lib.lynx_sparsify
-    assert f(None, 128, 512, vp(P), vp(P), None, None) == lynx.LYNX_ERR_INVALID_ARG
-    assert f(vp(P), 128, 500, vp(P), vp(P), None, None) == lynx.LYNX_ERR_UNSUPPORTED_SHAPE
-    assert f(vp(P), 128, 512, vp(P + 4), vp(P), None, None) == lynx.LYNX_ERR_MISALIGNED
-    assert f(vp(P), 128, 512, vp(P), vp(P), vp(P + 2), None) == lynx.LYNX_ERR_MISALIGNED
+    big = 1 << 30
+    assert f(None, 128, 512, vp(P), vp(P), None, vp(P), big, None) == lynx.LYNX_ERR_INVALID_ARG
+    assert f(vp(P), 128, 512, vp(P), vp(P), None, None, big, None) == lynx.LYNX_ERR_INVALID_ARG
+    assert f(vp(P), 128, 500, vp(P), vp(P), None, vp(P), big, None) == \
+        lynx.LYNX_ERR_UNSUPPORTED_SHAPE
+    assert f(vp(P), 128, 512, vp(P + 4), vp(P), None, vp(P), big, None) == lynx.LYNX_ERR_MISALIGNED
+    assert f(vp(P), 128, 512, vp(P), vp(P), vp(P + 2), vp(P), big, None) == \
+        lynx.LYNX_ERR_MISALIGNED
+    need = lynx.lynx_sparsify_workspace_bytes(128, 512)
+    assert need >= 8 * 128 * 8
+    assert f(vp(P), 128, 512, vp(P), vp(P), None, vp(P), need - 1, None) == \
+        lynx.LYNX_ERR_WORKSPACE_TOO_SMALL
 
 
 def test_sparse_gemm_argument_errors(lib):

@@ -193,26 +193,40 @@ def test_linear_is_deterministic():
     assert np.array_equal(y1, y2)
 
 
-def test_workspace_holds_sx_and_t():
+def check_workspace(ws, inp, rows=None):
+    """lynx_linear leaves in its workspace: the uncompensated kept values (exact
+    copies of X), the metadata, s per row and T/s.  Checked on `rows`."""
+    X = inp["X"]
+    M, K = X.shape
+    vals, meta, scale, t = helpers.workspace_views(ws.cpu().numpy(), M, K)
+    rows = np.arange(M) if rows is None else rows
+    canon = helpers.canonical_from_hw(meta, M, K)[rows]
+    ref = oracle.sparsify(X[rows])
+    assert np.array_equal(canon, ref["meta"])
+    assert np.array_equal(vals[rows], helpers.kept_from_x(X[rows], canon, K))
+    assert np.allclose(scale[rows], ref["scale"], rtol=4e-6, atol=0)
+    _, t_ref, _ = oracle.linear(X[rows], inp["W"][:8], None, inp["A"], inp["B"][:8])
+    s64 = ref["scale"].astype(np.float64)[:, None]
+    t_over_s = t_ref / s64
+    T = helpers.f32(t[rows]).astype(np.float64)
+    # T/s rounded once to bf16 (2^-9 relative, plus the division) on top of a
+    # K-term fp32 tensor-core accumulation, whose error is bounded by K * 2^-24
+    # times the sum of |x_k a_k| (<= 2^-10 of it for K <= 16384)
+    xa = np.abs(helpers.f32(X[rows]).astype(np.float64)) @ \
+        np.abs(helpers.f32(inp["A"]).astype(np.float64)).T
+    bound = 2 ** -8 * np.abs(t_over_s) + 2 ** -10 * xa / s64
+    ratio = np.abs(T - t_over_s) / bound
+    assert ratio.max() <= 1.0, f"T/s off: worst {ratio.max():.3g} of the bound"
+
+
+def test_workspace_holds_kept_values_scale_and_t():
     inp = workloads.make_linear_inputs(200, 576, 64, seed=17)
     M, K = inp["X"].shape
     ws = torch.zeros(lynx.lynx_workspace_bytes(M, 64, K, 64), dtype=torch.uint8, device=DEV)
     lynx.lynx_linear(dev(inp["X"]), dev(inp["W"]), dev(inp["bias"]), dev(inp["A"]),
                      dev(inp["B"]), workspace=ws)
     torch.cuda.synchronize()
-    raw = ws.cpu().numpy()
-    vals = raw[: M * K].view(np.uint16).reshape(M, K // 2)
-    meta_off = (M * K + 255) // 256 * 256
-    meta = raw[meta_off: meta_off + lynx.lynx_meta_bytes(M, K)]
-    ref = oracle.sparsify(inp["X"])
-    assert np.array_equal(helpers.canonical_from_hw(meta, M, K), ref["meta"])
-    assert helpers.bf16_ulp_distance(vals, ref["vals"]).max() <= 1
-    t_off = (meta_off + lynx.lynx_meta_bytes(M, K) + 255) // 256 * 256
-    t_off = (t_off + 4 * M + 255) // 256 * 256
-    T = helpers.f32(raw[t_off: t_off + M * 128].view(np.uint16).reshape(M, 64)).astype(np.float64)
-    _, t_ref, _ = oracle.linear(inp["X"], inp["W"], inp["bias"], inp["A"], inp["B"])
-    # bf16 rounding of an fp32-accumulated dot product
-    assert np.all(np.abs(T - t_ref) <= 2 ** -8 * np.abs(t_ref) + 1e-6)
+    check_workspace(ws, inp)
 
 
 # ---------------------------------------------------------------------------
@@ -233,14 +247,7 @@ def test_full_size_sampled_rows(name):
     args = [dev(inp[k]) for k in ("X", "W", "bias", "A", "B")]
     lynx.lynx_linear(*args, workspace=ws)
     torch.cuda.synchronize()
-    raw = ws.cpu().numpy()
-    vals = raw[: M * K].view(np.uint16).reshape(M, K // 2)
-    meta_off = (M * K + 255) // 256 * 256
-    meta = raw[meta_off: meta_off + lynx.lynx_meta_bytes(M, K)]
-    canon = helpers.canonical_from_hw(meta, M, K)
-    ref = oracle.sparsify(inp["X"][rows])
-    assert np.array_equal(canon[rows], ref["meta"])
-    assert helpers.bf16_ulp_distance(vals[rows], ref["vals"]).max() <= 1
+    check_workspace(ws, inp, rows=rows)
 
 
 # ---------------------------------------------------------------------------
@@ -269,3 +276,16 @@ def test_device_timeout_is_reported_and_context_survives():
     assert st == lynx.LYNX_OK and code == 0
     # the context is still usable and the next call is correct
     check_sparsify(X, *run_sparsify(X))
+
+
+def test_device_timeout_in_the_fused_layer():
+    inp = workloads.make_linear_inputs(256, 512, 256, seed=6)
+    args = [dev(inp[k]) for k in ("X", "W", "bias", "A", "B")]
+    lynx.lynx_debug_set_stall(True)
+    try:
+        lynx.lynx_linear(*args)
+        st, code = lynx.lynx_check_error()
+    finally:
+        lynx.lynx_debug_set_stall(False)
+    assert st == lynx.LYNX_ERR_DEVICE_TIMEOUT and code != 0
+    check_linear(inp)
