@@ -1,0 +1,359 @@
+// gemm_pair_kernel.cu -- the Lynx GEMM on CTA pairs (tcgen05 cta_group::2):
+//   Y[M,N] = bf16( s_row * (S(X) W^T + T' B^T) + bias )
+// Same arithmetic as gemm_kernel.cu (see there and the RT-Lynx references),
+// computed on 256 x 256 output tiles by a pair of CTAs on the two SMs of a
+// TPC: each CTA holds 128 rows of A (compressed activations, or X on the dense
+// path) and 128 of the 256 rows of the W tile in its own shared memory; one
+// tcgen05.mma(.sp).cta_group::2 with M = 256, N = 256 issued by the leader CTA
+// reads both halves, and each CTA's TMEM receives its 128 rows of the
+// accumulator.  Splitting B across the pair halves the operand bytes each SM
+// must stage per MMA, which is what the 2:4 sparse rate (twice the dense rate
+// per byte of B) needs.
+//
+// Per CTA (both CTAs run the same roles):
+//   warp 0      TMA producer: own 128 rows of A (and of the LoRA T), own 128
+//               rows of W (and of the LoRA B); on the sparse path one 2 KB
+//               metadata block (own 128 rows) every second stage.  All loads
+//               complete on the leader's "full" barrier (cta_group::2 form, no
+//               multicast); the leader arms it with both CTAs' bytes.
+//   warp 1      TMEM (pair allocation, 512 columns); in the leader CTA the
+//               single MMA issuer: tcgen05.cp of both CTAs' metadata, the MMAs,
+//               and commits multicast to both CTAs' "empty" / "acc_full"
+//               barriers.
+//   warps 2-9   epilogue on the CTA's own 128 accumulator rows: s * acc + bias
+//               -> bf16 -> global; releases the accumulator by arriving on the
+//               leader's "acc_empty" barrier.
+#include <cuda_bf16.h>
+
+#include "lynx_internal.h"
+#include "lynx_ptx.cuh"
+
+namespace lynx {
+
+namespace {
+
+constexpr int kThreads = 320;
+constexpr uint32_t kTmemCols = 512;
+constexpr int kGroupM = 8;  // pair-rows per raster group
+constexpr int kEslots = 4;
+constexpr uint32_t kBarEpilogue = 2;
+constexpr uint32_t kEpiThreads = 256;
+constexpr uint16_t kPairMask = 0x3;
+
+template <bool SPARSE>
+struct PairCfg {
+  static constexpr uint32_t kABytes = SPARSE ? 128u * 64u : 128u * 128u;  // own rows, one k-step
+  static constexpr uint32_t kBBytes = 128u * 128u;                        // own 128 W rows x 64 K
+  static constexpr uint32_t kEBytes = SPARSE ? 2048u : 0u;
+  static constexpr uint32_t kStageBytes = ((kABytes + kBBytes + kEBytes + 1023u) / 1024u) * 1024u;
+  static constexpr int kStagesFit = static_cast<int>((210u * 1024u) / kStageBytes);
+  static constexpr int kStages = kStagesFit > 8 ? 8 : kStagesFit;
+  static constexpr uint32_t kEcol0 = 256;
+  static constexpr uint32_t kLoraABytes = 128u * 64u;  // T: own 128 rows x 32
+  static constexpr uint32_t kLoraBBytes = 128u * 64u;  // B: own 128 rows x 32
+  static_assert(kStages >= 4, "pipeline too shallow");
+};
+
+template <bool SPARSE>
+struct __align__(1024) PairSmem {
+  using C = PairCfg<SPARSE>;
+  uint8_t stage[C::kStages][C::kStageBytes];
+  uint64_t full[C::kStages];   // used in the leader CTA
+  uint64_t empty[C::kStages];  // each CTA's producer waits on its own
+  uint64_t acc_full;           // each CTA's epilogue waits on its own
+  uint64_t acc_empty;          // used in the leader CTA (both CTAs' epilogues arrive)
+  uint64_t drain;
+  float bias_s[256];
+  uint32_t tmem_base;
+  volatile uint32_t abort_flag;
+};
+
+__device__ __forceinline__ void pair_tile_coords(int tile, int ntm2, int ntn, int& pm, int& nb) {
+  const int per_group = kGroupM * ntn;
+  const int group = tile / per_group;
+  const int first = group * kGroupM;
+  const int gm = min(kGroupM, ntm2 - first);
+  const int in_group = tile - group * per_group;
+  pm = first + in_group % gm;
+  nb = in_group / gm;
+}
+
+template <bool SPARSE>
+__global__ void __launch_bounds__(kThreads, 1)
+lynx_gemm_pair_kernel(const __grid_constant__ GemmLaunch p) {
+  using C = PairCfg<SPARSE>;
+  extern __shared__ uint8_t smem_raw[];
+  PairSmem<SPARSE>& sm = *reinterpret_cast<PairSmem<SPARSE>*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+
+  const uint32_t warp = warp_id_sync();
+  const uint32_t lane = lane_id();
+  const uint32_t rank = cluster_ctarank();  // 0 = leader of the pair
+  const bool leader = rank == 0;
+  const int ntm2 = static_cast<int>((p.M + 255) / 256);
+  const int ntn = static_cast<int>((p.N + 255) / 256);
+  const int ntiles = ntm2 * ntn;
+  const int cluster_id = static_cast<int>(blockIdx.x >> 1);
+  const int nclusters = static_cast<int>(gridDim.x >> 1);
+  const int nk = static_cast<int>(p.K / 64);
+  const int kblocks = static_cast<int>((p.K + 127) / 128);
+  const bool lora = p.lora != 0;
+  const int steps = nk + (lora ? 2 : 0);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::kStages; ++s) {
+      mbar_init(&sm.full[s], 1);
+      mbar_init(&sm.empty[s], 1);
+    }
+    mbar_init(&sm.acc_full, 1);
+    mbar_init(&sm.acc_empty, 2 * 8);
+    mbar_init(&sm.drain, 1);
+    sm.abort_flag = 0u;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(&sm.tmem_base, kTmemCols);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();  // both CTAs' barriers and TMEM exist before any cross-CTA signal
+  tc_fence_after();
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer (both CTAs)
+    if (lane == 0) {
+      tma_prefetch_desc(&p.tm_a);
+      tma_prefetch_desc(&p.tm_b);
+      if (SPARSE) tma_prefetch_desc(&p.tm_e);
+      if (lora) {
+        tma_prefetch_desc(&p.tm_t);
+        tma_prefetch_desc(&p.tm_lb);
+      }
+      uint32_t g = 0;
+      bool ok = !p.stall_test;
+      for (int tile = cluster_id; ok && tile < ntiles; tile += nclusters) {
+        int pm, nb;
+        pair_tile_coords(tile, ntm2, ntn, pm, nb);
+        const int32_t row0 = pm * 256 + static_cast<int32_t>(rank) * 128;
+        const int32_t col0 = nb * 256 + static_cast<int32_t>(rank) * 128;
+        const int mb = pm * 2 + static_cast<int>(rank);  // this CTA's 128-row block
+        for (int kit = 0; kit < steps; ++kit, ++g) {
+          const uint32_t slot = g % C::kStages;
+          const uint32_t ph = (g / C::kStages) & 1u;
+          if (sm.abort_flag || !mbar_wait(&sm.empty[slot], ph ^ 1u)) {
+            if (!sm.abort_flag) {
+              record_error(p.status, kDevTimeoutEmpty);
+              sm.abort_flag = 1u;
+            }
+            ok = false;
+            break;
+          }
+          uint8_t* st = sm.stage[slot];
+          const uint32_t lead_full = mapa_shared(smem_u32(&sm.full[slot]), 0);
+          if (kit < nk) {
+            const bool load_e = SPARSE && (kit % 2 == 0);
+            if (leader)
+              mbar_arrive_expect_tx(&sm.full[slot],
+                                    2u * (C::kABytes + C::kBBytes + (load_e ? 2048u : 0u)));
+            tma_load_2d_pair(st, &p.tm_a, lead_full, SPARSE ? kit * 32 : kit * 64, row0);
+            tma_load_2d_pair(st + C::kABytes, &p.tm_b, lead_full, kit * 64, col0);
+            if (load_e)
+              tma_load_2d_pair(st + C::kABytes + C::kBBytes, &p.tm_e, lead_full, 0,
+                               (mb * kblocks + kit / 2) * 128);
+          } else {
+            const int l = kit - nk;
+            if (leader) mbar_arrive_expect_tx(&sm.full[slot], 2u * (C::kLoraABytes + C::kLoraBBytes));
+            tma_load_2d_pair(st, &p.tm_t, lead_full, l * 32, row0);
+            tma_load_2d_pair(st + C::kABytes, &p.tm_lb, lead_full, l * 32, col0);
+          }
+        }
+      }
+      // drain (leader): the last fill of every stage, both CTAs' bytes, has landed
+      if (leader) {
+        const uint32_t issued = g;
+        for (uint32_t b = issued; b > 0 && b + C::kStages > issued; --b) {
+          const uint32_t x = b - 1;
+          if (!mbar_wait(&sm.full[x % C::kStages], (x / C::kStages) & 1u, kWaitLimitNs / 4))
+            record_error(p.status, kDevTimeoutDrain);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer (leader)
+    if (leader && lane == 0) {
+      const uint32_t idesc_main = make_idesc_bf16(256, 256, SPARSE);
+      const uint32_t idesc_dense = make_idesc_bf16(256, 256, false);
+      uint32_t g = 0, eslot = 0;
+      int acc_count = 0;
+      bool ok = true;
+      for (int tile = cluster_id; ok && tile < ntiles; tile += nclusters, ++acc_count) {
+        if (sm.abort_flag || !mbar_wait(&sm.acc_empty, (static_cast<uint32_t>(acc_count) & 1u) ^ 1u)) {
+          if (!sm.abort_flag) {
+            record_error(p.status, kDevTimeoutAccum);
+            sm.abort_flag = 1u;
+          }
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = sm.tmem_base;
+        uint32_t accumulate = 0;
+        for (int kit = 0; kit < steps; ++kit, ++g) {
+          const uint32_t slot = g % C::kStages;
+          const uint32_t ph = (g / C::kStages) & 1u;
+          if (sm.abort_flag || !mbar_wait(&sm.full[slot], ph)) {
+            if (!sm.abort_flag) {
+              record_error(p.status, kDevTimeoutFull);
+              sm.abort_flag = 1u;
+            }
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sa = smem_u32(sm.stage[slot]);
+          const uint32_t sb = sa + C::kABytes;
+          if (kit < nk) {
+            if (SPARSE) {
+              if (kit % 2 == 0) {
+                eslot = (eslot + 1) % kEslots;
+                const uint64_t edesc = make_sdesc(sb + C::kBBytes, 2048, 128, kSwNone);
+                tc_cp_128x128b_pair(sm.tmem_base + C::kEcol0 + 4 * eslot, edesc);
+              }
+#pragma unroll
+              for (int j = 0; j < 2; ++j) {
+                const uint32_t ecol = C::kEcol0 + 4 * eslot + 2 * (kit % 2) + j;
+                const uint64_t da = make_sdesc(sa + 32 * j, 16, 512, kSw64);
+                const uint64_t db = make_sdesc(sb + 64 * j, 16, 1024, kSw128);
+                mma_sp_bf16_pair(d_tmem, da, db, sm.tmem_base + (ecol & ~1u), idesc_main | (ecol & 1u),
+                                 accumulate);
+                accumulate = 1;
+              }
+            } else {
+#pragma unroll
+              for (int kk = 0; kk < 4; ++kk) {
+                const uint64_t da = make_sdesc(sa + 32 * kk, 16, 1024, kSw128);
+                const uint64_t db = make_sdesc(sb + 32 * kk, 16, 1024, kSw128);
+                mma_bf16_pair(d_tmem, da, db, idesc_main, accumulate);
+                accumulate = 1;
+              }
+            }
+          } else {
+#pragma unroll
+            for (int kk = 0; kk < 2; ++kk) {
+              const uint64_t da = make_sdesc(sa + 32 * kk, 16, 512, kSw64);
+              const uint64_t db = make_sdesc(sb + 32 * kk, 16, 512, kSw64);
+              mma_bf16_pair(d_tmem, da, db, idesc_dense, accumulate);
+              accumulate = 1;
+            }
+          }
+          tc_commit_pair_mc(&sm.empty[slot], kPairMask);
+        }
+        if (!ok) break;
+        tc_commit_pair_mc(&sm.acc_full, kPairMask);
+      }
+      tc_commit_pair_mc(&sm.drain, 0x1);
+      if (!mbar_wait(&sm.drain, 0)) record_error(p.status, kDevTimeoutDrain);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ epilogue (both CTAs)
+    constexpr int kHalf = 128;                 // columns per warp
+    const uint32_t q = warp & 3u;              // TMEM lane quarter this warp may access
+    const uint32_t ch = (warp - 2u) >> 2;      // which half of the 256 columns
+    const uint32_t row = 32u * q + lane;
+    const uint32_t et = threadIdx.x - 64u;     // 0..255
+    const __nv_bfloat16* bias = static_cast<const __nv_bfloat16*>(p.bias);
+    __nv_bfloat16* y = static_cast<__nv_bfloat16*>(p.y);
+    const uint32_t lead_acc_empty = mapa_shared(smem_u32(&sm.acc_empty), 0);
+    int acc_count = 0;
+    for (int tile = cluster_id; tile < ntiles; tile += nclusters, ++acc_count) {
+      int pm, nb;
+      pair_tile_coords(tile, ntm2, ntn, pm, nb);
+      const int64_t grow = static_cast<int64_t>(pm) * 256 + rank * 128 + row;
+      const bool row_ok = grow < p.M;
+      const int64_t n_base = static_cast<int64_t>(nb) * 256;
+      named_bar_sync(kBarEpilogue, kEpiThreads);  // the previous tile's bias is no longer read
+      {
+        const int64_t n = n_base + et;
+        sm.bias_s[et] = (bias != nullptr && n < p.N) ? __bfloat162float(bias[n]) : 0.f;
+      }
+      const float s = (p.row_scale != nullptr && row_ok) ? p.row_scale[grow] : 1.f;
+      bool ok = !sm.abort_flag;
+      if (ok && !mbar_wait(&sm.acc_full, static_cast<uint32_t>(acc_count) & 1u)) {
+        record_error(p.status, kDevTimeoutAccum);
+        sm.abort_flag = 1u;
+        ok = false;
+      }
+      if (named_bar_red_or(kBarEpilogue, kEpiThreads, !ok)) break;
+      tc_fence_after();
+      uint32_t out[kHalf / 2];
+#pragma unroll
+      for (int c = 0; c < kHalf / 32; ++c) {
+        const int col = static_cast<int>(ch) * kHalf + 32 * c;
+        uint32_t r[32];
+        tmem_ld_32x32b_x32(sm.tmem_base + ((32u * q) << 16) + static_cast<uint32_t>(col), r);
+        tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const float a = __fmaf_rn(s, __uint_as_float(r[2 * i]), sm.bias_s[col + 2 * i]);
+          const float b = __fmaf_rn(s, __uint_as_float(r[2 * i + 1]), sm.bias_s[col + 2 * i + 1]);
+          __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+          out[16 * c + i] = *reinterpret_cast<uint32_t*>(&h);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(lead_acc_empty);
+      if (row_ok) {
+        const int64_t n0 = n_base + static_cast<int64_t>(ch) * kHalf;
+        __nv_bfloat16* yrow = y + grow * p.N + n0;
+#pragma unroll
+        for (int v = 0; v < kHalf / 8; ++v) {
+          if (n0 + 8 * v < p.N)
+            *reinterpret_cast<uint4*>(yrow + 8 * v) =
+                make_uint4(out[4 * v], out[4 * v + 1], out[4 * v + 2], out[4 * v + 3]);
+        }
+      }
+    }
+  }
+
+  __syncthreads();
+  cluster_sync_all();  // the pair's MMAs, copies and epilogues are all finished
+  if (warp == 1) tmem_dealloc_pair(sm.tmem_base, kTmemCols);
+}
+
+template <bool SPARSE>
+cudaError_t launch_pair_variant(const GemmLaunch& p, cudaStream_t stream) {
+  const size_t smem = sizeof(PairSmem<SPARSE>) + 1024;
+  static int configured_device = -1;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (configured_device != dev) {
+    cudaError_t e = cudaFuncSetAttribute(lynx_gemm_pair_kernel<SPARSE>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    configured_device = dev;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(p.grid), 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, lynx_gemm_pair_kernel<SPARSE>, p);
+}
+
+}  // namespace
+
+cudaError_t launch_gemm_pair(const GemmLaunch& p, cudaStream_t stream) {
+  return p.sparse ? launch_pair_variant<true>(p, stream) : launch_pair_variant<false>(p, stream);
+}
+
+}  // namespace lynx

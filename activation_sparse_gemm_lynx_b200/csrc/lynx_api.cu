@@ -145,26 +145,35 @@ lynx_status run_sparsify(DeviceState* ds, const void* X, const void* A, int64_t 
   return map_cuda(launch_sparsify(p, stream));
 }
 
+// CTA pairs (256 x 256 tiles) unless the problem is too small to feed them
+bool use_pair_kernel(int64_t M, int64_t N) { return M > 128 && N >= 256; }
+
 lynx_status run_gemm(DeviceState* ds, const void* a_src, bool sparse, const void* meta,
                      const float* row_scale, const void* T, const void* W, const void* bias,
                      const void* B, int64_t M, int64_t N, int64_t K, void* Y, cudaStream_t stream) {
   GemmLaunch p;
   std::memset(&p, 0, sizeof(p));
-  const int bn = gemm_bn(N);
+  const bool pair = use_pair_kernel(M, N);
+  const int bn = pair ? 256 : gemm_bn(N);
+  const uint32_t b_rows = pair ? 128u : static_cast<uint32_t>(bn);  // W rows one CTA loads
   if (sparse) {
     if (!encode_bf16_2d(&p.tm_a, a_src, K / 2, M, K, 32, 128, CU_TENSOR_MAP_SWIZZLE_64B))
+      return LYNX_ERR_CUDA;
+    if (pair && !encode_u8_2d(&p.tm_e, meta, 16,
+                              static_cast<uint64_t>(meta_row_blocks(M)) * ((K + 127) / 128) * 128, 16,
+                              16, 128))
       return LYNX_ERR_CUDA;
   } else {
     if (!encode_bf16_2d(&p.tm_a, a_src, K, M, K * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B))
       return LYNX_ERR_CUDA;
   }
-  if (!encode_bf16_2d(&p.tm_b, W, K, N, K * 2, 64, bn, CU_TENSOR_MAP_SWIZZLE_128B))
+  if (!encode_bf16_2d(&p.tm_b, W, K, N, K * 2, 64, b_rows, CU_TENSOR_MAP_SWIZZLE_128B))
     return LYNX_ERR_CUDA;
   const bool lora = (T != nullptr && B != nullptr);
   if (lora) {
     if (!encode_bf16_2d(&p.tm_t, T, kLoraRank, M, kLoraRank * 2, 32, 128, CU_TENSOR_MAP_SWIZZLE_64B))
       return LYNX_ERR_CUDA;
-    if (!encode_bf16_2d(&p.tm_lb, B, kLoraRank, N, kLoraRank * 2, 32, bn, CU_TENSOR_MAP_SWIZZLE_64B))
+    if (!encode_bf16_2d(&p.tm_lb, B, kLoraRank, N, kLoraRank * 2, 32, b_rows, CU_TENSOR_MAP_SWIZZLE_64B))
       return LYNX_ERR_CUDA;
   }
   p.meta = static_cast<const uint8_t*>(meta);
@@ -177,10 +186,16 @@ lynx_status run_gemm(DeviceState* ds, const void* a_src, bool sparse, const void
   p.sparse = sparse ? 1 : 0;
   p.lora = lora ? 1 : 0;
   p.bn = bn;
-  const int64_t tiles = ((M + 127) / 128) * ((N + bn - 1) / bn);
-  p.grid = static_cast<int>(tiles < ds->sms ? tiles : ds->sms);
   p.stall_test = g_stall.load();
   p.status = ds->status;
+  if (pair) {
+    const int64_t tiles = ((M + 255) / 256) * ((N + 255) / 256);
+    const int64_t pairs = ds->sms / 2;
+    p.grid = static_cast<int>(2 * (tiles < pairs ? tiles : pairs));
+    return map_cuda(launch_gemm_pair(p, stream));
+  }
+  const int64_t tiles = ((M + 127) / 128) * ((N + bn - 1) / bn);
+  p.grid = static_cast<int>(tiles < ds->sms ? tiles : ds->sms);
   return map_cuda(launch_gemm(p, stream));
 }
 
@@ -197,6 +212,20 @@ bool encode_bf16_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t
   cuuint32_t estr[2] = {1, 1};
   CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
                         strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+bool encode_u8_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer,
+                  uint64_t row_pitch_bytes, uint32_t box_inner, uint32_t box_outer) {
+  std::call_once(g_encode_once, resolve_encode);
+  if (g_encode == nullptr) return false;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {row_pitch_bytes};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims,
+                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
@@ -236,7 +265,7 @@ size_t lynx_vals_bytes(int64_t M, int64_t K) {
 
 size_t lynx_meta_bytes(int64_t M, int64_t K) {
   if (M <= 0 || K <= 0) return 0;
-  return static_cast<size_t>((M + 127) / 128) * static_cast<size_t>((K + 127) / 128) *
+  return static_cast<size_t>(meta_row_blocks(M)) * static_cast<size_t>((K + 127) / 128) *
          static_cast<size_t>(kMetaBlockBytes);
 }
 
@@ -394,7 +423,7 @@ int lynx_meta_canonical_to_hw(const uint8_t* canonical, uint8_t* hw, int64_t M, 
   if (hw == nullptr || canonical == nullptr) return LYNX_ERR_INVALID_ARG;
   if (M < 1 || K < 8 || K % 8 != 0) return LYNX_ERR_UNSUPPORTED_SHAPE;
   const int64_t kblocks = (K + 127) / 128;
-  const int64_t mpad = (M + 127) / 128 * 128;
+  const int64_t mpad = meta_row_blocks(M) * 128;
   std::memset(hw, 0, lynx_meta_bytes(M, K));
   for (int64_t m = 0; m < mpad; ++m) {
     for (int64_t g = 0; g < K / 4; ++g) {

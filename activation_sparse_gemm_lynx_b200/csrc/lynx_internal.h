@@ -53,6 +53,7 @@ struct GemmLaunch {
   CUtensorMap tm_b;     // W [N,K] box 64 x BN, SW128
   CUtensorMap tm_t;     // T [M,64] box 32 x 128, SW64 (lora)
   CUtensorMap tm_lb;    // B [N,64] box 32 x BN, SW64 (lora)
+  CUtensorMap tm_e;     // metadata as uint8 [blocks*128, 16], box 16 x 128 (pair kernel)
   const uint8_t* meta;  // hardware metadata blocks (sparse)
   const void* bias;     // [N] bf16 or null
   const float* row_scale;  // [M] fp32 multiplier of each accumulator row, or null
@@ -66,9 +67,17 @@ struct GemmLaunch {
   uint32_t* status;
 };
 
-cudaError_t launch_gemm(const GemmLaunch& p, cudaStream_t stream);
+cudaError_t launch_gemm(const GemmLaunch& p, cudaStream_t stream);       // 128 x BN tiles, 1 CTA
+cudaError_t launch_gemm_pair(const GemmLaunch& p, cudaStream_t stream);  // 256 x 256 tiles, CTA pairs
 
 // ---- helpers ----------------------------------------------------------------
+
+// 128-row blocks of metadata are allocated in pairs (a CTA pair covers 256 rows)
+inline int64_t meta_row_blocks(int64_t M) { return (M + 255) / 256 * 2; }
+
+// 2-D uint8 tensor map (no swizzle)
+bool encode_u8_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer,
+                  uint64_t row_pitch_bytes, uint32_t box_inner, uint32_t box_outer);
 
 // 2-D bf16 tensor map: inner (contiguous) extent, outer extent, row pitch in bytes
 bool encode_bf16_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer,

@@ -276,7 +276,7 @@ sparsify_kernel(const __grid_constant__ SparsifyLaunch p) {
       }
       if (ct == 0) bulk_wait_read_all();  // the store of tile b-1 has read its buffer
       stop = named_bar_red_or(kBarCompute, kComputeThreads, !ok);
-      if (!stop && ct == 0) {
+      if (!stop && ct == 0 && mb * 128 < p.M) {
         tma_store_2d(&p.tm_vals, sm.vstage[b & 1], static_cast<int32_t>((kcol0 + 64 * b) / 2),
                      static_cast<int32_t>(mb * 128));
         bulk_commit();
@@ -388,7 +388,7 @@ size_t sparsify_smem_bytes() { return sizeof(SparsifySmem) + 1024; }
 // K ranges per row block: the largest C <= kMaxSplit dividing the 64-column
 // boxes of a row such that C * ceil(M/128) CTAs fit in one wave (2 per SM).
 int choose_sparsify_split(int64_t M, int64_t K, int num_sms) {
-  const int64_t row_blocks = (M + 127) / 128;
+  const int64_t row_blocks = meta_row_blocks(M);
   const int64_t boxes = K / 64;
   int best = 1;
   for (int c = 2; c <= kMaxSplit; ++c) {
@@ -410,7 +410,9 @@ cudaError_t launch_sparsify(const SparsifyLaunch& p, cudaStream_t stream) {
     if (e != cudaSuccess) return e;
     configured_device = dev;
   }
-  const dim3 grid(static_cast<unsigned>(p.split), static_cast<unsigned>((p.M + 127) / 128), 1);
+  // metadata row blocks come in pairs: the block past M (if any) gets the
+  // pattern of all-zero rows, so a CTA pair of the GEMM never reads garbage
+  const dim3 grid(static_cast<unsigned>(p.split), static_cast<unsigned>(meta_row_blocks(p.M)), 1);
   sparsify_kernel<<<grid, kThreads, smem, stream>>>(p);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;

@@ -81,13 +81,15 @@ LYNX_API int lynx_lora_rank(void);
 LYNX_API size_t lynx_vals_bytes(int64_t M, int64_t K);
 
 /* Bytes of the 2:4 metadata in the tcgen05.mma.sp operand layout: one
- * 2048-byte block per 128 rows x 128 dense K, rows padded to a multiple of 128
- * and K to a multiple of 128: ceil(M/128) * ceil(K/128) * 2048.
+ * 2048-byte block per 128 rows x 128 dense K; rows are padded to a multiple of
+ * 256 (128-row blocks come in pairs, one per CTA of a CTA pair) and K to a
+ * multiple of 128: ceil(M/256) * 2 * ceil(K/128) * 2048.
  * Layout: block (mb, kb) at byte (mb * ceil(K/128) + kb) * 2048; inside a
  * block, row m and dense column k (both relative to the block) map to TMEM
  * lane L = (m % 8) + 8 * ((k / 16) % 2) + 16 * (m / 16), 32-bit word
  * w = k / 32 of the lane's 16 bytes, bit b = (k % 16) + 16 * ((m / 8) % 2);
- * each group of 4 owns 4 bits: lo | hi << 2 (lo < hi its kept positions). */
+ * each group of 4 owns 4 bits: lo | hi << 2 (lo < hi its kept positions).
+ * Padding rows hold the pattern of an all-zero row (lo = 0, hi = 1). */
 LYNX_API size_t lynx_meta_bytes(int64_t M, int64_t K);
 
 /* Bytes of the workspace lynx_linear needs (kept values, metadata, row scales,
@@ -106,7 +108,7 @@ LYNX_API size_t lynx_sparsify_workspace_bytes(int64_t M, int64_t K);
  *   vals      [M,K/2] bf16, out: kept values after compensation, two per group,
  *             ascending position (lynx_vals_bytes)
  *   meta      out: metadata blocks, lynx_meta_bytes(M,K) bytes (layout above);
- *             rows M..ceil(M/128)*128-1 hold the pattern of an all-zero row
+ *             padding rows hold the pattern of an all-zero row
  *   row_scale [M] fp32, out: s per row, or NULL
  *   workspace caller-allocated scratch of workspace_bytes >=
  *             lynx_sparsify_workspace_bytes(M,K) */

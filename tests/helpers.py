@@ -44,7 +44,7 @@ def canonical_from_hw(hw, M, K):
 def hw_from_canonical(canon, M, K):
     """Canonical [M, K/8] -> hardware bytes (padding rows: pattern of a zero row)."""
     kblocks = (K + 127) // 128
-    mpad = (M + 127) // 128 * 128
+    mpad = (M + 255) // 256 * 256   # 128-row blocks come in pairs
     out = np.zeros(mpad // 128 * kblocks * 2048, dtype=np.uint8)
     full = np.full((mpad, K // 8), 0x44, dtype=np.uint8)
     full[:M] = canon
@@ -109,7 +109,7 @@ def workspace_views(raw, M, K, r=64):
     def a256(x):
         return (x + 255) // 256 * 256
     kblocks = (K + 127) // 128
-    meta_bytes = (M + 127) // 128 * kblocks * 2048
+    meta_bytes = (M + 255) // 256 * 2 * kblocks * 2048
     o_meta = a256(M * K)
     o_scale = a256(o_meta + meta_bytes)
     o_t = a256(o_scale + 4 * M)

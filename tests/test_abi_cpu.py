@@ -38,7 +38,7 @@ def test_status_strings(lib):
 @pytest.mark.parametrize("M,K", [(1, 64), (128, 128), (129, 192), (4608, 3072), (4608, 12288)])
 def test_sizes(lib, M, K):
     assert lynx.lynx_vals_bytes(M, K) == M * K
-    assert lynx.lynx_meta_bytes(M, K) == -(-M // 128) * -(-K // 128) * 2048
+    assert lynx.lynx_meta_bytes(M, K) == -(-M // 256) * 2 * -(-K // 128) * 2048
     ws = lynx.lynx_workspace_bytes(M, 512, K, 64)
     assert ws >= M * K + lynx.lynx_meta_bytes(M, K) + 4 * M + 128 * M
     assert ws % 256 == 0
@@ -126,7 +126,7 @@ def test_meta_padding_rows_hold_zero_row_pattern(lib):
     M, K = 130, 256
     canon = np.full((M, K // 8), 0xEE, dtype=np.uint8)   # (2,3) everywhere
     hw = lynx.lynx_meta_canonical_to_hw(canon, M + 0, K)
-    pad = helpers.canonical_from_hw(hw, 256, K)[M:]
+    pad = helpers.canonical_from_hw(hw, 256, K)[M:]  # padded to 256 rows
     assert np.all(pad == 0x44)
 
 
