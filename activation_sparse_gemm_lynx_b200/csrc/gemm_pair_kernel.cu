@@ -13,7 +13,7 @@
 // Per CTA (both CTAs run the same roles):
 //   warp 0      TMA producer: own 128 rows of A (and of the LoRA T), own 128
 //               rows of W (and of the LoRA B); on the sparse path one 2 KB
-//               metadata block (own 128 rows) every second stage.  All loads
+//               metadata block (own 128 rows) per stage.  All loads
 //               complete on the leader's "full" barrier (cta_group::2 form, no
 //               multicast); the leader arms it with both CTAs' bytes.
 //   warp 1      TMEM (pair allocation, 512 columns); in the leader CTA the
@@ -34,19 +34,24 @@ namespace {
 
 constexpr int kThreads = 320;
 constexpr uint32_t kTmemCols = 512;
-constexpr int kGroupM = 8;  // pair-rows per raster group
 constexpr int kEslots = 4;
 constexpr uint32_t kBarEpilogue = 2;
 constexpr uint32_t kEpiThreads = 256;
 constexpr uint16_t kPairMask = 0x3;
 
+// One pipeline stage covers kBK dense K: 128 on the sparse path (A: 128 rows x
+// 64 kept values = one 128-byte-row tile; W: two 128 x 64 tiles; one 2 KB
+// metadata block), 64 on the dense path.  LoRA stages (K = 32 each) reuse the
+// A / B slots with 64-byte-row tiles.
 template <bool SPARSE>
 struct PairCfg {
-  static constexpr uint32_t kABytes = SPARSE ? 128u * 64u : 128u * 128u;  // own rows, one k-step
-  static constexpr uint32_t kBBytes = 128u * 128u;                        // own 128 W rows x 64 K
+  static constexpr int kBK = SPARSE ? 128 : 64;
+  static constexpr uint32_t kABytes = 128u * 128u;                            // 16 KB: own 128 rows
+  static constexpr uint32_t kBBytes = 128u * static_cast<uint32_t>(kBK) * 2u;  // own 128 W rows
   static constexpr uint32_t kEBytes = SPARSE ? 2048u : 0u;
   static constexpr uint32_t kStageBytes = ((kABytes + kBBytes + kEBytes + 1023u) / 1024u) * 1024u;
-  static constexpr int kStagesFit = static_cast<int>((210u * 1024u) / kStageBytes);
+  // of the 227 KB: 16 KB epilogue store staging, ~3 KB barriers / bias / alignment
+  static constexpr int kStagesFit = static_cast<int>((208u * 1024u) / kStageBytes);
   static constexpr int kStages = kStagesFit > 8 ? 8 : kStagesFit;
   static constexpr uint32_t kEcol0 = 256;
   static constexpr uint32_t kLoraABytes = 128u * 64u;  // T: own 128 rows x 32
@@ -58,6 +63,7 @@ template <bool SPARSE>
 struct __align__(1024) PairSmem {
   using C = PairCfg<SPARSE>;
   uint8_t stage[C::kStages][C::kStageBytes];
+  uint8_t ystage[8][2][1024];  // per epilogue warp: two 32 rows x 16 columns bf16 tiles (32B swizzle)
   uint64_t full[C::kStages];   // used in the leader CTA
   uint64_t empty[C::kStages];  // each CTA's producer waits on its own
   uint64_t acc_full;           // each CTA's epilogue waits on its own
@@ -68,11 +74,14 @@ struct __align__(1024) PairSmem {
   volatile uint32_t abort_flag;
 };
 
-__device__ __forceinline__ void pair_tile_coords(int tile, int ntm2, int ntn, int& pm, int& nb) {
-  const int per_group = kGroupM * ntn;
+// tiles walk M first inside a group of `group_m` pair-rows (sized on the host so
+// that the group's A rows stay resident in L2 while W streams once per group)
+__device__ __forceinline__ void pair_tile_coords(int tile, int ntm2, int ntn, int group_m, int& pm,
+                                                 int& nb) {
+  const int per_group = group_m * ntn;
   const int group = tile / per_group;
-  const int first = group * kGroupM;
-  const int gm = min(kGroupM, ntm2 - first);
+  const int first = group * group_m;
+  const int gm = min(group_m, ntm2 - first);
   const int in_group = tile - group * per_group;
   pm = first + in_group % gm;
   nb = in_group / gm;
@@ -95,7 +104,7 @@ lynx_gemm_pair_kernel(const __grid_constant__ GemmLaunch p) {
   const int ntiles = ntm2 * ntn;
   const int cluster_id = static_cast<int>(blockIdx.x >> 1);
   const int nclusters = static_cast<int>(gridDim.x >> 1);
-  const int nk = static_cast<int>(p.K / 64);
+  const int nk = static_cast<int>(p.K / C::kBK);
   const int kblocks = static_cast<int>((p.K + 127) / 128);
   const bool lora = p.lora != 0;
   const int steps = nk + (lora ? 2 : 0);
@@ -134,7 +143,7 @@ lynx_gemm_pair_kernel(const __grid_constant__ GemmLaunch p) {
       bool ok = !p.stall_test;
       for (int tile = cluster_id; ok && tile < ntiles; tile += nclusters) {
         int pm, nb;
-        pair_tile_coords(tile, ntm2, ntn, pm, nb);
+        pair_tile_coords(tile, ntm2, ntn, p.group_m, pm, nb);
         const int32_t row0 = pm * 256 + static_cast<int32_t>(rank) * 128;
         const int32_t col0 = nb * 256 + static_cast<int32_t>(rank) * 128;
         const int mb = pm * 2 + static_cast<int>(rank);  // this CTA's 128-row block
@@ -152,15 +161,16 @@ lynx_gemm_pair_kernel(const __grid_constant__ GemmLaunch p) {
           uint8_t* st = sm.stage[slot];
           const uint32_t lead_full = mapa_shared(smem_u32(&sm.full[slot]), 0);
           if (kit < nk) {
-            const bool load_e = SPARSE && (kit % 2 == 0);
-            if (leader)
-              mbar_arrive_expect_tx(&sm.full[slot],
-                                    2u * (C::kABytes + C::kBBytes + (load_e ? 2048u : 0u)));
-            tma_load_2d_pair(st, &p.tm_a, lead_full, SPARSE ? kit * 32 : kit * 64, row0);
-            tma_load_2d_pair(st + C::kABytes, &p.tm_b, lead_full, kit * 64, col0);
-            if (load_e)
+            if (leader) mbar_arrive_expect_tx(&sm.full[slot], 2u * (C::kABytes + C::kBBytes + C::kEBytes));
+            // A: 64 kept values (sparse) or 64 dense values (dense) per row
+            tma_load_2d_pair(st, &p.tm_a, lead_full, kit * 64, row0);
+            tma_load_2d_pair(st + C::kABytes, &p.tm_b, lead_full, kit * C::kBK, col0);
+            if (SPARSE) {
+              tma_load_2d_pair(st + C::kABytes + 16384, &p.tm_b, lead_full, kit * C::kBK + 64, col0);
+              // metadata block (mb, kit): 2 KB seen as 8 rows of 256 bytes
               tma_load_2d_pair(st + C::kABytes + C::kBBytes, &p.tm_e, lead_full, 0,
-                               (mb * kblocks + kit / 2) * 128);
+                               (mb * kblocks + kit) * 8);
+            }
           } else {
             const int l = kit - nk;
             if (leader) mbar_arrive_expect_tx(&sm.full[slot], 2u * (C::kLoraABytes + C::kLoraBBytes));
@@ -181,15 +191,19 @@ lynx_gemm_pair_kernel(const __grid_constant__ GemmLaunch p) {
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer (leader)
-    if (leader && lane == 0) {
+    // The whole warp runs the loop (operands stay warp-uniform); one elected
+    // lane issues each tcgen05 instruction.
+    if (leader) {
       const uint32_t idesc_main = make_idesc_bf16(256, 256, SPARSE);
       const uint32_t idesc_dense = make_idesc_bf16(256, 256, false);
       uint32_t g = 0, eslot = 0;
       int acc_count = 0;
       bool ok = true;
       for (int tile = cluster_id; ok && tile < ntiles; tile += nclusters, ++acc_count) {
-        if (sm.abort_flag || !mbar_wait(&sm.acc_empty, (static_cast<uint32_t>(acc_count) & 1u) ^ 1u)) {
-          if (!sm.abort_flag) {
+        bool got = !sm.abort_flag && mbar_wait(&sm.acc_empty, (static_cast<uint32_t>(acc_count) & 1u) ^ 1u);
+        got = __all_sync(0xffffffffu, got);
+        if (!got) {
+          if (!sm.abort_flag && lane == 0) {
             record_error(p.status, kDevTimeoutAccum);
             sm.abort_flag = 1u;
           }
@@ -201,8 +215,10 @@ lynx_gemm_pair_kernel(const __grid_constant__ GemmLaunch p) {
         for (int kit = 0; kit < steps; ++kit, ++g) {
           const uint32_t slot = g % C::kStages;
           const uint32_t ph = (g / C::kStages) & 1u;
-          if (sm.abort_flag || !mbar_wait(&sm.full[slot], ph)) {
-            if (!sm.abort_flag) {
+          bool ready = !sm.abort_flag && mbar_wait(&sm.full[slot], ph);
+          ready = __all_sync(0xffffffffu, ready);
+          if (!ready) {
+            if (!sm.abort_flag && lane == 0) {
               record_error(p.status, kDevTimeoutFull);
               sm.abort_flag = 1u;
             }
@@ -214,18 +230,19 @@ lynx_gemm_pair_kernel(const __grid_constant__ GemmLaunch p) {
           const uint32_t sb = sa + C::kABytes;
           if (kit < nk) {
             if (SPARSE) {
-              if (kit % 2 == 0) {
-                eslot = (eslot + 1) % kEslots;
-                const uint64_t edesc = make_sdesc(sb + C::kBBytes, 2048, 128, kSwNone);
-                tc_cp_128x128b_pair(sm.tmem_base + C::kEcol0 + 4 * eslot, edesc);
-              }
+              eslot = (eslot + 1) % kEslots;
+              const uint64_t edesc = make_sdesc(sb + C::kBBytes, 2048, 128, kSwNone);
+              if (elect_one()) tc_cp_128x128b_pair(sm.tmem_base + C::kEcol0 + 4 * eslot, edesc);
+              __syncwarp();
 #pragma unroll
-              for (int j = 0; j < 2; ++j) {
-                const uint32_t ecol = C::kEcol0 + 4 * eslot + 2 * (kit % 2) + j;
-                const uint64_t da = make_sdesc(sa + 32 * j, 16, 512, kSw64);
-                const uint64_t db = make_sdesc(sb + 64 * j, 16, 1024, kSw128);
-                mma_sp_bf16_pair(d_tmem, da, db, sm.tmem_base + (ecol & ~1u), idesc_main | (ecol & 1u),
-                                 accumulate);
+              for (int j = 0; j < 4; ++j) {
+                const uint32_t ecol = C::kEcol0 + 4 * eslot + j;
+                const uint64_t da = make_sdesc(sa + 32 * j, 16, 1024, kSw128);
+                const uint64_t db = make_sdesc(sb + (j >> 1) * 16384 + 64 * (j & 1), 16, 1024, kSw128);
+                if (elect_one())
+                  mma_sp_bf16_pair(d_tmem, da, db, sm.tmem_base + (ecol & ~1u), idesc_main | (ecol & 1u),
+                                   accumulate);
+                __syncwarp();
                 accumulate = 1;
               }
             } else {
@@ -233,7 +250,8 @@ lynx_gemm_pair_kernel(const __grid_constant__ GemmLaunch p) {
               for (int kk = 0; kk < 4; ++kk) {
                 const uint64_t da = make_sdesc(sa + 32 * kk, 16, 1024, kSw128);
                 const uint64_t db = make_sdesc(sb + 32 * kk, 16, 1024, kSw128);
-                mma_bf16_pair(d_tmem, da, db, idesc_main, accumulate);
+                if (elect_one()) mma_bf16_pair(d_tmem, da, db, idesc_main, accumulate);
+                __syncwarp();
                 accumulate = 1;
               }
             }
@@ -242,17 +260,21 @@ lynx_gemm_pair_kernel(const __grid_constant__ GemmLaunch p) {
             for (int kk = 0; kk < 2; ++kk) {
               const uint64_t da = make_sdesc(sa + 32 * kk, 16, 512, kSw64);
               const uint64_t db = make_sdesc(sb + 32 * kk, 16, 512, kSw64);
-              mma_bf16_pair(d_tmem, da, db, idesc_dense, accumulate);
+              if (elect_one()) mma_bf16_pair(d_tmem, da, db, idesc_dense, accumulate);
+              __syncwarp();
               accumulate = 1;
             }
           }
-          tc_commit_pair_mc(&sm.empty[slot], kPairMask);
+          if (elect_one()) tc_commit_pair_mc(&sm.empty[slot], kPairMask);
+          __syncwarp();
         }
         if (!ok) break;
-        tc_commit_pair_mc(&sm.acc_full, kPairMask);
+        if (elect_one()) tc_commit_pair_mc(&sm.acc_full, kPairMask);
+        __syncwarp();
       }
-      tc_commit_pair_mc(&sm.drain, 0x1);
-      if (!mbar_wait(&sm.drain, 0)) record_error(p.status, kDevTimeoutDrain);
+      if (elect_one()) tc_commit_pair_mc(&sm.drain, 0x1);
+      __syncwarp();
+      if (!mbar_wait(&sm.drain, 0) && lane == 0) record_error(p.status, kDevTimeoutDrain);
     }
     __syncwarp();
   } else {
@@ -263,12 +285,11 @@ lynx_gemm_pair_kernel(const __grid_constant__ GemmLaunch p) {
     const uint32_t row = 32u * q + lane;
     const uint32_t et = threadIdx.x - 64u;     // 0..255
     const __nv_bfloat16* bias = static_cast<const __nv_bfloat16*>(p.bias);
-    __nv_bfloat16* y = static_cast<__nv_bfloat16*>(p.y);
     const uint32_t lead_acc_empty = mapa_shared(smem_u32(&sm.acc_empty), 0);
     int acc_count = 0;
     for (int tile = cluster_id; tile < ntiles; tile += nclusters, ++acc_count) {
       int pm, nb;
-      pair_tile_coords(tile, ntm2, ntn, pm, nb);
+      pair_tile_coords(tile, ntm2, ntn, p.group_m, pm, nb);
       const int64_t grow = static_cast<int64_t>(pm) * 256 + rank * 128 + row;
       const bool row_ok = grow < p.M;
       const int64_t n_base = static_cast<int64_t>(nb) * 256;
@@ -286,35 +307,52 @@ lynx_gemm_pair_kernel(const __grid_constant__ GemmLaunch p) {
       }
       if (named_bar_red_or(kBarEpilogue, kEpiThreads, !ok)) break;
       tc_fence_after();
-      uint32_t out[kHalf / 2];
-#pragma unroll
+      // 32 columns at a time: TMEM -> registers -> s * acc + bias -> bf16 ->
+      // two 16-column pieces staged in shared memory -> asynchronous bulk
+      // tensor stores (rows past M / columns past N are clipped by the TMA)
+      const int32_t store_row = static_cast<int32_t>(pm * 256 + rank * 128 + 32 * q);
+      uint8_t* my_stage = sm.ystage[warp - 2][0];
+      int piece = 0;
+#pragma unroll 1
       for (int c = 0; c < kHalf / 32; ++c) {
         const int col = static_cast<int>(ch) * kHalf + 32 * c;
         uint32_t r[32];
         tmem_ld_32x32b_x32(sm.tmem_base + ((32u * q) << 16) + static_cast<uint32_t>(col), r);
         tmem_ld_wait();
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const float a = __fmaf_rn(s, __uint_as_float(r[2 * i]), sm.bias_s[col + 2 * i]);
-          const float b = __fmaf_rn(s, __uint_as_float(r[2 * i + 1]), sm.bias_s[col + 2 * i + 1]);
-          __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
-          out[16 * c + i] = *reinterpret_cast<uint32_t*>(&h);
+        if (c == kHalf / 32 - 1) {
+          // every TMEM read of this tile is done: hand the accumulator back
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive_cluster(lead_acc_empty);
         }
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(lead_acc_empty);
-      if (row_ok) {
-        const int64_t n0 = n_base + static_cast<int64_t>(ch) * kHalf;
-        __nv_bfloat16* yrow = y + grow * p.N + n0;
 #pragma unroll
-        for (int v = 0; v < kHalf / 8; ++v) {
-          if (n0 + 8 * v < p.N)
-            *reinterpret_cast<uint4*>(yrow + 8 * v) =
-                make_uint4(out[4 * v], out[4 * v + 1], out[4 * v + 2], out[4 * v + 3]);
+        for (int h = 0; h < 2; ++h, ++piece) {
+          uint32_t pk[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const int e = 16 * h + 2 * i;
+            const float a = __fmaf_rn(s, __uint_as_float(r[e]), sm.bias_s[col + e]);
+            const float b = __fmaf_rn(s, __uint_as_float(r[e + 1]), sm.bias_s[col + e + 1]);
+            __nv_bfloat162 hv = __floats2bfloat162_rn(a, b);
+            pk[i] = *reinterpret_cast<uint32_t*>(&hv);
+          }
+          uint8_t* buf = my_stage + 1024 * (piece & 1);
+          if (lane == 0) bulk_wait_read_le1();  // the store that last used `buf` has read it
+          __syncwarp();
+          // row `lane`, 16-byte chunks k = 0,1 at 32B-swizzled positions
+          const uint32_t sw = (lane >> 2) & 1u;
+          *reinterpret_cast<uint4*>(buf + lane * 32 + ((0u ^ sw) << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          *reinterpret_cast<uint4*>(buf + lane * 32 + ((1u ^ sw) << 4)) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_2d(&p.tm_y, buf, static_cast<int32_t>(n_base + col + 16 * h), store_row);
+            bulk_commit();
+          }
         }
       }
     }
+    if (lane == 0) bulk_wait_all();  // every Y tile this warp issued is written
   }
 
   __syncthreads();

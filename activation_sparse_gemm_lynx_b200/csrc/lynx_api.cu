@@ -145,23 +145,29 @@ lynx_status run_sparsify(DeviceState* ds, const void* X, const void* A, int64_t 
   return map_cuda(launch_sparsify(p, stream));
 }
 
-// CTA pairs (256 x 256 tiles) unless the problem is too small to feed them
-bool use_pair_kernel(int64_t M, int64_t N) { return M > 128 && N >= 256; }
+// CTA pairs (256 x 256 tiles) unless the problem is too small to feed them; the
+// sparse pair kernel steps K by 128
+bool use_pair_kernel(int64_t M, int64_t N, int64_t K, bool sparse) {
+  return M > 128 && N >= 256 && (!sparse || K % 128 == 0);
+}
 
 lynx_status run_gemm(DeviceState* ds, const void* a_src, bool sparse, const void* meta,
                      const float* row_scale, const void* T, const void* W, const void* bias,
                      const void* B, int64_t M, int64_t N, int64_t K, void* Y, cudaStream_t stream) {
   GemmLaunch p;
   std::memset(&p, 0, sizeof(p));
-  const bool pair = use_pair_kernel(M, N);
+  const bool pair = use_pair_kernel(M, N, K, sparse);
   const int bn = pair ? 256 : gemm_bn(N);
   const uint32_t b_rows = pair ? 128u : static_cast<uint32_t>(bn);  // W rows one CTA loads
   if (sparse) {
-    if (!encode_bf16_2d(&p.tm_a, a_src, K / 2, M, K, 32, 128, CU_TENSOR_MAP_SWIZZLE_64B))
+    // pair kernel: 128-byte rows of 64 kept values; single-CTA kernel: 64-byte rows
+    if (!encode_bf16_2d(&p.tm_a, a_src, K / 2, M, K, pair ? 64 : 32, 128,
+                        pair ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B))
       return LYNX_ERR_CUDA;
-    if (pair && !encode_u8_2d(&p.tm_e, meta, 16,
-                              static_cast<uint64_t>(meta_row_blocks(M)) * ((K + 127) / 128) * 128, 16,
-                              16, 128))
+    // metadata blocks of 2 KB seen as 8 rows of 256 bytes
+    if (pair && !encode_u8_2d(&p.tm_e, meta, 256,
+                              static_cast<uint64_t>(meta_row_blocks(M)) * ((K + 127) / 128) * 8, 256,
+                              256, 8))
       return LYNX_ERR_CUDA;
   } else {
     if (!encode_bf16_2d(&p.tm_a, a_src, K, M, K * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B))
@@ -176,6 +182,8 @@ lynx_status run_gemm(DeviceState* ds, const void* a_src, bool sparse, const void
     if (!encode_bf16_2d(&p.tm_lb, B, kLoraRank, N, kLoraRank * 2, 32, b_rows, CU_TENSOR_MAP_SWIZZLE_64B))
       return LYNX_ERR_CUDA;
   }
+  if (pair && !encode_bf16_2d(&p.tm_y, Y, N, M, N * 2, 16, 32, CU_TENSOR_MAP_SWIZZLE_32B))
+    return LYNX_ERR_CUDA;
   p.meta = static_cast<const uint8_t*>(meta);
   p.row_scale = row_scale;
   p.bias = bias;
@@ -189,13 +197,21 @@ lynx_status run_gemm(DeviceState* ds, const void* a_src, bool sparse, const void
   p.stall_test = g_stall.load();
   p.status = ds->status;
   if (pair) {
-    const int64_t tiles = ((M + 255) / 256) * ((N + 255) / 256);
+    const int64_t ntm2 = (M + 255) / 256;
+    const int64_t tiles = ntm2 * ((N + 255) / 256);
     const int64_t pairs = ds->sms / 2;
     p.grid = static_cast<int>(2 * (tiles < pairs ? tiles : pairs));
+    // raster group: as many 256-row pair-rows of A as fit in ~40 MB of L2, so
+    // the group's A stays resident while W streams once per group
+    const int64_t a_row_bytes = 256 * (sparse ? K : 2 * K);
+    int64_t gm = (40ll << 20) / (a_row_bytes > 0 ? a_row_bytes : 1);
+    gm = gm < 1 ? 1 : (gm > ntm2 ? ntm2 : gm);
+    p.group_m = static_cast<int>(gm);
     return map_cuda(launch_gemm_pair(p, stream));
   }
   const int64_t tiles = ((M + 127) / 128) * ((N + bn - 1) / bn);
   p.grid = static_cast<int>(tiles < ds->sms ? tiles : ds->sms);
+  p.group_m = 16;
   return map_cuda(launch_gemm(p, stream));
 }
 

@@ -53,7 +53,8 @@ struct GemmLaunch {
   CUtensorMap tm_b;     // W [N,K] box 64 x BN, SW128
   CUtensorMap tm_t;     // T [M,64] box 32 x 128, SW64 (lora)
   CUtensorMap tm_lb;    // B [N,64] box 32 x BN, SW64 (lora)
-  CUtensorMap tm_e;     // metadata as uint8 [blocks*128, 16], box 16 x 128 (pair kernel)
+  CUtensorMap tm_e;     // metadata as uint8 [blocks*8, 256], box 256 x 8 (pair kernel)
+  CUtensorMap tm_y;     // Y [M,N] bf16, box 16 x 32, 32B swizzle (pair kernel stores)
   const uint8_t* meta;  // hardware metadata blocks (sparse)
   const void* bias;     // [N] bf16 or null
   const float* row_scale;  // [M] fp32 multiplier of each accumulator row, or null
@@ -63,6 +64,7 @@ struct GemmLaunch {
   int lora;
   int bn;               // 128 or 256
   int grid;             // persistent CTAs
+  int group_m;          // tile rows (of 128 or of 256 for CTA pairs) per raster group
   int stall_test;
   uint32_t* status;
 };

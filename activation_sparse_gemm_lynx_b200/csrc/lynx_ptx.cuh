@@ -43,6 +43,17 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
 
 __device__ __forceinline__ uint32_t lane_id() { return threadIdx.x & 31u; }
 
+// one lane of the (fully active) warp returns true; the others false.  Used to
+// issue tcgen05 / TMA instructions from a warp whose every lane computes the
+// same operands, which keeps those operands in warp-uniform registers.
+__device__ __forceinline__ bool elect_one() {
+  uint32_t p;
+  asm volatile(
+      "{\n\t.reg .pred P;\n\telect.sync _|P, 0xffffffff;\n\tselp.u32 %0, 1, 0, P;\n\t}"
+      : "=r"(p));
+  return p != 0;
+}
+
 __device__ __forceinline__ uint32_t warp_id_sync() {
   return __shfl_sync(0xffffffffu, threadIdx.x >> 5, 0);
 }
@@ -151,6 +162,12 @@ __device__ __forceinline__ void bulk_commit() {
 // all committed bulk stores of this thread have finished reading shared memory
 __device__ __forceinline__ void bulk_wait_read_all() {
   asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+
+// at most one committed bulk store group of this thread may still be reading
+// shared memory
+__device__ __forceinline__ void bulk_wait_read_le1() {
+  asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
 }
 
 // all committed bulk stores of this thread are complete
