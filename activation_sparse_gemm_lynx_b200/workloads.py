@@ -111,6 +111,22 @@ def make_config_inputs(name: str, **kw) -> dict:
     return make_linear_inputs(c.M, c.K, c.N, c.r, seed=c.seed, x_kind=c.x_kind, **kw)
 
 
+def make_rank_inputs(name: str, rank: int, **kw) -> dict:
+    """One data-parallel rank's inputs of a named workload.
+
+    Token rows are independent, so the layer shards by rows: every rank holds
+    the same W, bias, A and B (the config's own draws) and its own batch of
+    activations.  Rank 0's batch is the config's X; rank q > 0 draws a fresh X
+    of the same shape and kind from the seed ``[config seed, q]``.
+    """
+    c = CONFIGS[name]
+    inp = make_config_inputs(name, **kw)
+    if rank > 0:
+        rng = np.random.default_rng([c.seed, rank])
+        inp["X"] = f32_to_bf16_bits(draw_activations(rng, c.M, c.K, c.x_kind))
+    return inp
+
+
 def sweep_skip_blocks() -> list:
     """The 2 of 8 blocks whose linears are left dense (selective layer skipping)."""
     rng = np.random.default_rng(SWEEP_SEED)

@@ -35,10 +35,20 @@ sys.path.insert(0, ROOT)
 METRIC = "sparse-act linear dense-equiv TFLOP/s (2MNK/t) & speedup vs dense bf16 GEMM"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
-# DRAM bytes (read + write) per launch of the sparse GEMM kernel from one ncu
-# capture of the same kernel, per workload; None until captured for the kernel
-# as it stands (see profiles/).
-GEMM_DRAM_TRAFFIC = {}
+# DRAM bytes (read + write) per launch of the sparse GEMM kernel, from one ncu
+# capture of the kernel as it stands (dram__bytes_read.sum + dram__bytes_write.sum);
+# a workload that has not been captured reports null.
+GEMM_DRAM_TRAFFIC = {"mlp_up": 93.97e6 + 83.43e6}
+
+# kernels one sparse lynx_linear call launches: sparsify pass, per-row finalize, GEMM
+LAUNCHES_PER_LINEAR = 3
+
+
+def gemm_kernel_name(M, N, K):
+    """Name of the GEMM kernel the library picks for a sparse call of this shape."""
+    if M > 128 and N >= 256 and K % 128 == 0:
+        return "lynx_gemm_pair_kernel<1> (CTA pair, 256x256 tiles)"
+    return f"lynx_gemm_kernel<{256 if N >= 1024 else 128},1>"
 
 
 def parse_args(argv=None):
@@ -88,16 +98,16 @@ def max_over_ranks(value, world):
     return float(t.item())
 
 
+def aggregate_tflops(flops_per_rank, ms_max, world):
+    """Whole-job throughput: the work of all ranks over the slowest rank's time."""
+    return world * flops_per_rank / (ms_max * 1e-3) / 1e12
+
+
 def barrier(world):
     if world > 1:
         import torch.distributed as dist
 
         dist.barrier()
-
-
-def rank_seed(base_seed, rank):
-    """Each rank draws its own batch of the workload (same shapes)."""
-    return base_seed if rank == 0 else [base_seed, rank]
 
 
 # ---------------------------------------------------------------------------
@@ -272,8 +282,7 @@ def run_lynx(args):
 
     shape = workloads.CONFIGS[args.workload]
     M, N, K, r = shape.M, shape.N, shape.K, shape.r
-    inp = workloads.make_linear_inputs(M, K, N, r, seed=rank_seed(shape.seed, rank),
-                                       x_kind=shape.x_kind)
+    inp = workloads.make_rank_inputs(args.workload, rank)
 
     def dev(a):
         return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).cuda()
@@ -383,7 +392,7 @@ def run_lynx(args):
 
     result = {
         "metric": METRIC,
-        "value": world * flops / (ms_step * 1e-3) / 1e12,
+        "value": aggregate_tflops(flops, ms_step, world),
         "unit": "TFLOP/s",
         "n_gpus": world,
         "steps": args.steps,
@@ -404,7 +413,7 @@ def run_lynx(args):
         "breakdown_ms": {"linear": ms_step, "sparsify_pass": sp_ms, "sparse_gemm": gemm_ms,
                          "dense_torch_matmul": dense_ms, "lynx_dense_path": lynx_dense_ms},
         "roofline": {
-            "bound": "tensor", "kernel": "lynx_gemm_kernel<256,sparse>",
+            "bound": "tensor", "kernel": gemm_kernel_name(M, N, K),
             "achieved": gemm_tflops, "peak": sparse_peak, "unit": "TFLOP/s",
             "frac": gemm_tflops / sparse_peak, "traffic": traffic,
             "peak_note": f"2 x {peaks['source']} dense bf16 burst ({peaks['bf16_tflops']} TFLOP/s); "
@@ -417,12 +426,12 @@ def run_lynx(args):
             "traffic": None,
             "work": "X read 2MK + vals MK + meta MK/8 + T 2Mr + s 4M + A 2rK bytes",
         },
-        "e2e": {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+        "e2e": {"value": aggregate_tflops(flops, e2e_ms, world), "unit": "TFLOP/s",
                 "h2d_bytes_per_step": 2 * M * K, "d2h_bytes_per_step": 2 * M * N,
                 "ms_per_step": e2e_ms,
                 "note": "X copied from pinned host memory and Y copied back inside each step; "
                         "weights resident"},
-        "gpu_launches": 2 * args.steps,
+        "gpu_launches": LAUNCHES_PER_LINEAR * args.steps,
         "clocks": clock_info,
     }
 
