@@ -25,6 +25,8 @@ from .lynx import (  # noqa: F401
     lynx_profile_set_split_event,
     lynx_sparse_gemm,
     lynx_sparsify,
+    lynx_sparsify_noalloc,
+    lynx_sparsify_noalloc_max_rows,
     lynx_sparsify_workspace_bytes,
     lynx_status_string,
     lynx_vals_bytes,

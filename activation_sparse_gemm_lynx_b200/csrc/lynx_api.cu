@@ -13,6 +13,12 @@
 // Per-device status word: the first error code a kernel records wins.
 static __device__ uint32_t g_lynx_status_word;
 
+// Scratch of lynx_sparsify_noalloc: per-split partial row sums, then s (when
+// the caller gives no row_scale buffer).  Sized for LYNX_SPARSIFY_NOALLOC_MAX_ROWS.
+constexpr size_t kNoAllocLpartBytes = size_t(8) * LYNX_SPARSIFY_NOALLOC_MAX_ROWS * 8;
+constexpr size_t kNoAllocScratchBytes = kNoAllocLpartBytes + size_t(LYNX_SPARSIFY_NOALLOC_MAX_ROWS) * 4;
+static __device__ __align__(256) unsigned char g_sparsify_noalloc_scratch[kNoAllocScratchBytes];
+
 namespace lynx {
 
 namespace {
@@ -53,6 +59,26 @@ DeviceState* device_state() {
     if (d.err == cudaSuccess) d.err = cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev);
   });
   return d.err == cudaSuccess ? &d : nullptr;
+}
+
+// Device address of this device's noalloc scratch, looked up once per device.
+struct NoAllocState {
+  std::once_flag once;
+  uint8_t* scratch = nullptr;
+  cudaError_t err = cudaSuccess;
+};
+NoAllocState g_noalloc[kMaxDevices];
+
+uint8_t* noalloc_scratch() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  NoAllocState& st = g_noalloc[dev];
+  std::call_once(st.once, [&st]() {
+    void* p = nullptr;
+    st.err = cudaGetSymbolAddress(&p, g_sparsify_noalloc_scratch);
+    if (st.err == cudaSuccess) st.scratch = static_cast<uint8_t*>(p);
+  });
+  return st.err == cudaSuccess ? st.scratch : nullptr;
 }
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -313,6 +339,28 @@ int lynx_sparsify(const void* X, int64_t M, int64_t K, void* vals, void* meta, f
   float* scale = row_scale ? row_scale : reinterpret_cast<float*>(ws + wl.scale);
   return run_sparsify(ds, X, nullptr, M, K, vals, meta, scale, nullptr,
                       reinterpret_cast<float2*>(ws + wl.lpart), nullptr, kModeSelect | kModeScaled,
+                      static_cast<cudaStream_t>(stream));
+}
+
+int64_t lynx_sparsify_noalloc_max_rows(void) { return LYNX_SPARSIFY_NOALLOC_MAX_ROWS; }
+
+int lynx_sparsify_noalloc(const void* X, int64_t M, int64_t K, void* vals, void* meta,
+                          float* row_scale, void* stream) {
+  static_assert(kMaxSplit == 8, "noalloc scratch is sized for 8 K-splits");
+  if (X == nullptr || vals == nullptr || meta == nullptr) return LYNX_ERR_INVALID_ARG;
+  lynx_status st = check_shape(M, 0, K);
+  if (st != LYNX_OK) return st;
+  if (M > LYNX_SPARSIFY_NOALLOC_MAX_ROWS) return LYNX_ERR_WORKSPACE_TOO_SMALL;
+  if (!aligned16(X) || !aligned16(vals) || !aligned16(meta) ||
+      (reinterpret_cast<uintptr_t>(row_scale) & 3u) != 0)
+    return LYNX_ERR_MISALIGNED;
+  DeviceState* ds = device_state();
+  if (ds == nullptr) return LYNX_ERR_CUDA;
+  uint8_t* scratch = noalloc_scratch();
+  if (scratch == nullptr) return LYNX_ERR_CUDA;
+  float* scale = row_scale ? row_scale : reinterpret_cast<float*>(scratch + kNoAllocLpartBytes);
+  return run_sparsify(ds, X, nullptr, M, K, vals, meta, scale, nullptr,
+                      reinterpret_cast<float2*>(scratch), nullptr, kModeSelect | kModeScaled,
                       static_cast<cudaStream_t>(stream));
 }
 

@@ -53,6 +53,8 @@ def library():
             "lynx_workspace_bytes": ([i64, i64, i64, i64], sz),
             "lynx_sparsify_workspace_bytes": ([i64, i64], sz),
             "lynx_sparsify": ([p, i64, i64, p, p, p, p, sz, p], i32),
+            "lynx_sparsify_noalloc": ([p, i64, i64, p, p, p, p], i32),
+            "lynx_sparsify_noalloc_max_rows": ([], i64),
             "lynx_linear": ([p, p, p, p, p, i64, i64, i64, i64, i32, p, p, sz, p], i32),
             "lynx_linear_dense": ([p, p, p, p, p, i64, i64, i64, i64, p, p, sz, p], i32),
             "lynx_sparse_gemm": ([p, p, p, p, p, p, i64, i64, i64, i64, p, p], i32),
@@ -164,6 +166,29 @@ def lynx_sparsify(X, vals=None, meta=None, row_scale=None, workspace=None, strea
     st = library().lynx_sparsify(_ptr(X), M, K, _ptr(vals), _ptr(meta), _ptr(row_scale),
                                  _ptr(workspace), workspace.numel(), _stream(stream))
     _check(st, "lynx_sparsify")
+    return vals, meta, row_scale
+
+
+def lynx_sparsify_noalloc_max_rows():
+    return library().lynx_sparsify_noalloc_max_rows()
+
+
+def lynx_sparsify_noalloc(X, vals, meta, row_scale=None, stream=None):
+    """S(X) into caller buffers, with the library's fixed scratch instead of a
+    workspace; allocates nothing.  Returns (vals, meta, row_scale)."""
+    import torch
+
+    _need(X, "X", torch.bfloat16)
+    M, K = X.shape
+    _need(vals, "vals", torch.bfloat16, (M, K // 2))
+    _need(meta, "meta", torch.uint8)
+    if meta.numel() < lynx_meta_bytes(M, K):
+        raise ValueError("meta buffer too small")
+    if row_scale is not None:
+        _need(row_scale, "row_scale", torch.float32, (M,))
+    st = library().lynx_sparsify_noalloc(_ptr(X), M, K, _ptr(vals), _ptr(meta), _ptr(row_scale),
+                                         _stream(stream))
+    _check(st, "lynx_sparsify_noalloc")
     return vals, meta, row_scale
 
 

@@ -116,6 +116,37 @@ LYNX_API int lynx_sparsify(const void* X, int64_t M, int64_t K, void* vals, void
                            float* row_scale, void* workspace, size_t workspace_bytes,
                            void* stream);
 
+/* ---- S(X) without a caller workspace ---------------------------------- */
+
+/* Largest M lynx_sparsify_noalloc accepts. */
+#define LYNX_SPARSIFY_NOALLOC_MAX_ROWS 16384
+
+/* lynx_sparsify with its scratch (the per-range partial row sums and, when
+ * row_scale is NULL, s) in a fixed device array of the library instead of a
+ * caller workspace: LYNX_SPARSIFY_NOALLOC_MAX_ROWS * (8 * 8 + 4) bytes
+ * (1.06 MiB) per device.  The RT-Lynx pages have no counterpart of this entry
+ * point; it exists for callers that cannot hand out a workspace: code behind a
+ * fixed operator signature that receives only its inputs and outputs, and
+ * latency-critical loops that must not call cudaMalloc (which can synchronise
+ * the whole device) nor go through another runtime's allocator.
+ *   Arguments, output layout, results and errors are those of lynx_sparsify.
+ *   M > LYNX_SPARSIFY_NOALLOC_MAX_ROWS returns LYNX_ERR_WORKSPACE_TOO_SMALL
+ *   before anything is launched.
+ *   The call allocates no memory.  The first call on a device looks up the
+ *   scratch's device address (cudaGetSymbolAddress) and the device's SM count;
+ *   make that first call before any stream capture.
+ *   Nothing in the scratch has to start at zero: every call writes all the
+ *   partials it reads.
+ *   All calls on one device share the one scratch array: two calls whose device
+ *   work overlaps (different streams, or different host threads, without an
+ *   ordering between them) race on it and give wrong results.  Calls in order
+ *   on one stream are safe. */
+LYNX_API int lynx_sparsify_noalloc(const void* X, int64_t M, int64_t K, void* vals, void* meta,
+                                   float* row_scale, void* stream);
+
+/* LYNX_SPARSIFY_NOALLOC_MAX_ROWS, for callers without the header. */
+LYNX_API int64_t lynx_sparsify_noalloc_max_rows(void);
+
 /* Y = S(X) W^T + bias + (X A^T) B^T  (S(X) = X when skip_sparsify != 0).
  *   X [M,K], W [N,K] (frozen backbone weight), bias [N] or NULL,
  *   A [r,K] and B [N,r] (LoRA, both or neither; r must be 64), Y [M,N] out.
