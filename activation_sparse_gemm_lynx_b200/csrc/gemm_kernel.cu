@@ -115,6 +115,9 @@ lynx_gemm_kernel(const __grid_constant__ GemmLaunch p) {
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  // the prologue above may overlap the previous kernel (programmatic launch);
+  // its outputs are read only from here on
+  pdl_wait();
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -337,8 +340,8 @@ cudaError_t launch_variant(const GemmLaunch& p, cudaStream_t stream) {
     if (e != cudaSuccess) return e;
     configured_device = dev;
   }
-  lynx_gemm_kernel<BN, SPARSE><<<p.grid, kGemmThreads, smem, stream>>>(p);
-  return cudaGetLastError();
+  return launch_after_previous(lynx_gemm_kernel<BN, SPARSE>, dim3(static_cast<unsigned>(p.grid)),
+                               dim3(kGemmThreads), smem, stream, p);
 }
 
 }  // namespace

@@ -128,6 +128,9 @@ lynx_gemm_pair_kernel(const __grid_constant__ GemmLaunch p) {
   __syncthreads();
   cluster_sync_all();  // both CTAs' barriers and TMEM exist before any cross-CTA signal
   tc_fence_after();
+  // the prologue above may overlap the previous kernel (programmatic launch);
+  // its outputs (compressed values, metadata, s, T) are read only from here on
+  pdl_wait();
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer (both CTAs)
@@ -307,32 +310,33 @@ lynx_gemm_pair_kernel(const __grid_constant__ GemmLaunch p) {
       }
       if (named_bar_red_or(kBarEpilogue, kEpiThreads, !ok)) break;
       tc_fence_after();
-      // 32 columns at a time: TMEM -> registers -> s * acc + bias -> bf16 ->
-      // two 16-column pieces staged in shared memory -> asynchronous bulk
+      // The warp's 32 rows x 128 columns of the accumulator go to registers
+      // first and the accumulator is handed back at once, so the next tile's
+      // MMAs start while this tile is converted and stored: s * acc + bias ->
+      // bf16 -> 16-column pieces staged in shared memory -> asynchronous bulk
       // tensor stores (rows past M / columns past N are clipped by the TMA)
       const int32_t store_row = static_cast<int32_t>(pm * 256 + rank * 128 + 32 * q);
       uint8_t* my_stage = sm.ystage[warp - 2][0];
+      uint32_t r[kHalf / 32][32];
+#pragma unroll
+      for (int c = 0; c < kHalf / 32; ++c)
+        tmem_ld_32x32b_x32(sm.tmem_base + ((32u * q) << 16) + ch * kHalf + 32u * c, r[c]);
+      tmem_ld_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(lead_acc_empty);
       int piece = 0;
-#pragma unroll 1
+#pragma unroll
       for (int c = 0; c < kHalf / 32; ++c) {
         const int col = static_cast<int>(ch) * kHalf + 32 * c;
-        uint32_t r[32];
-        tmem_ld_32x32b_x32(sm.tmem_base + ((32u * q) << 16) + static_cast<uint32_t>(col), r);
-        tmem_ld_wait();
-        if (c == kHalf / 32 - 1) {
-          // every TMEM read of this tile is done: hand the accumulator back
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive_cluster(lead_acc_empty);
-        }
 #pragma unroll
         for (int h = 0; h < 2; ++h, ++piece) {
           uint32_t pk[8];
 #pragma unroll
           for (int i = 0; i < 8; ++i) {
             const int e = 16 * h + 2 * i;
-            const float a = __fmaf_rn(s, __uint_as_float(r[e]), sm.bias_s[col + e]);
-            const float b = __fmaf_rn(s, __uint_as_float(r[e + 1]), sm.bias_s[col + e + 1]);
+            const float a = __fmaf_rn(s, __uint_as_float(r[c][e]), sm.bias_s[col + e]);
+            const float b = __fmaf_rn(s, __uint_as_float(r[c][e + 1]), sm.bias_s[col + e + 1]);
             __nv_bfloat162 hv = __floats2bfloat162_rn(a, b);
             pk[i] = *reinterpret_cast<uint32_t*>(&hv);
           }
@@ -378,13 +382,15 @@ cudaError_t launch_pair_variant(const GemmLaunch& p, cudaStream_t stream) {
   cfg.blockDim = dim3(kThreads, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   return cudaLaunchKernelEx(&cfg, lynx_gemm_pair_kernel<SPARSE>, p);
 }
 

@@ -3,6 +3,7 @@
 #pragma once
 
 #include <cstdint>
+#include <utility>
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -42,6 +43,25 @@ struct SparsifyLaunch {
 };
 
 // sparsify pass + finalize (+ rescale for the standalone form), on one stream
+// Launches `kernel` with programmatic stream serialization: it may begin (and
+// run its prologue) while the previous kernel on `stream` finishes; it must call
+// pdl_wait() before it reads anything that kernel wrote.
+template <typename... Params, typename... Args>
+cudaError_t launch_after_previous(void (*kernel)(Params...), dim3 grid, dim3 block, size_t smem,
+                                  cudaStream_t stream, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
 cudaError_t launch_sparsify(const SparsifyLaunch& p, cudaStream_t stream);
 int choose_sparsify_split(int64_t M, int64_t K, int num_sms);
 size_t sparsify_smem_bytes();

@@ -54,6 +54,19 @@ __device__ __forceinline__ bool elect_one() {
   return p != 0;
 }
 
+// Programmatic dependent launch.  A kernel launched with programmatic stream
+// serialization may start while the previous kernel on the stream is still
+// running; pdl_wait() returns once that kernel has completed and its memory
+// operations are visible (a no-op without such a predecessor).  Every thread
+// that reads the predecessor's output calls it first.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// Lets the next kernel on the stream (if launched with programmatic stream
+// serialization) begin its launch; it still waits in pdl_wait() for this grid.
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 __device__ __forceinline__ uint32_t warp_id_sync() {
   return __shfl_sync(0xffffffffu, threadIdx.x >> 5, 0);
 }

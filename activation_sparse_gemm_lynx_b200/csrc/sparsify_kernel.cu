@@ -66,47 +66,47 @@ struct __align__(1024) SparsifySmem {
   uint64_t full[kStages];
   uint64_t empty[kStages];     // row threads done with a stage (one arrival per warp)
   uint64_t mma_done[kStages];  // the LoRA MMAs done with a stage (tcgen05.commit)
+  uint64_t vfree[2];           // a value staging buffer has been read by its TMA store
   uint64_t tdone;
   uint64_t drain;
   uint32_t tmem_base;
   volatile uint32_t abort_flag;
 };
 
-__device__ __forceinline__ uint64_t pack_f2(float lo, float hi) {
-  return static_cast<uint64_t>(__float_as_uint(lo)) |
-         (static_cast<uint64_t>(__float_as_uint(hi)) << 32);
-}
-
-// (a.x + b.x, a.y + b.y), each an IEEE fp32 add rounded to nearest even
-__device__ __forceinline__ uint64_t add_f32x2(uint64_t a, uint64_t b) {
-  uint64_t r;
-  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
-  return r;
-}
-
-// |x| of both bf16 halves of w, widened to fp32 (exact): (low half, high half)
-__device__ __forceinline__ uint64_t abs_pair(uint32_t w) {
-  const uint32_t a = w & 0x7FFF7FFFu;
-  return pack_f2(__uint_as_float(a << 16), __uint_as_float(a & 0xFFFF0000u));
+// acc_lo += |low bf16 of w|, acc_hi += |high bf16 of w|: each half widened to
+// fp32 exactly, the magnitude taken by the add's operand modifier
+__device__ __forceinline__ void add_abs_pair(float& acc_lo, float& acc_hi, uint32_t w) {
+  acc_lo = __fadd_rn(acc_lo, fabsf(__uint_as_float(w << 16)));
+  acc_hi = __fadd_rn(acc_hi, fabsf(__uint_as_float(w & 0xFFFF0000u)));
 }
 
 // Top-2 of the 4 bf16 values in (w0 = x1:x0, w1 = x3:x2) by magnitude, ties to
-// the lower index.  Each value becomes a distinct key (|x| << 2) | (3 - i), so a
-// larger key is a larger magnitude or, on equal magnitude, a lower index; the
-// two largest keys come out of a 4-input max/min network.  Returns the nibble
-// lo | hi << 2 and the kept pair packed (x_lo in the low half).
-__device__ __forceinline__ uint32_t select_group(uint32_t w0, uint32_t w1, uint32_t& kept) {
-  const uint32_t k0 = ((w0 << 2) & 0x1FFFCu) | 3u;
-  const uint32_t k1 = ((w0 >> 14) & 0x1FFFCu) | 2u;
-  const uint32_t k2 = ((w1 << 2) & 0x1FFFCu) | 1u;
-  const uint32_t k3 = ((w1 >> 14) & 0x1FFFCu);
+// the lower index, together with the group's terms of the row's L1 sum.  Each
+// value is widened to fp32 (exact); its magnitude bits with (3 - i) in the two
+// lowest bits form a distinct key, so a larger key is a larger magnitude or, on
+// equal magnitude, a lower index, and the two largest keys come out of a
+// 4-input max/min network.  Adds |x0|, |x2| to la_even and |x1|, |x3| to
+// la_odd; returns the nibble lo | hi << 2 and the kept pair packed (x_lo in the
+// low half).
+__device__ __forceinline__ uint32_t select_group(uint32_t w0, uint32_t w1, uint32_t& kept,
+                                                 float& la_even, float& la_odd) {
+  const uint32_t f0 = w0 << 16, f1 = w0 & 0xFFFF0000u;
+  const uint32_t f2 = w1 << 16, f3 = w1 & 0xFFFF0000u;
+  la_even = __fadd_rn(la_even, fabsf(__uint_as_float(f0)));
+  la_odd = __fadd_rn(la_odd, fabsf(__uint_as_float(f1)));
+  la_even = __fadd_rn(la_even, fabsf(__uint_as_float(f2)));
+  la_odd = __fadd_rn(la_odd, fabsf(__uint_as_float(f3)));
+  const uint32_t k0 = (f0 & 0x7FFF0000u) | 3u;
+  const uint32_t k1 = (f1 & 0x7FFF0000u) | 2u;
+  const uint32_t k2 = (f2 & 0x7FFF0000u) | 1u;
+  const uint32_t k3 = f3 & 0x7FFF0000u;
   const uint32_t p = max(k0, k1), q = min(k0, k1);
   const uint32_t r = max(k2, k3), u = min(k2, k3);
   const uint32_t t1 = max(p, r);
   const uint32_t t2 = max(min(p, r), max(q, u));
   const uint32_t a = t1 & 3u, b = t2 & 3u;  // 3 - index of the two winners
-  const uint32_t lo = 3u - max(a, b);
-  const uint32_t hi = 3u - min(a, b);
+  const uint32_t lo = 3u ^ max(a, b);
+  const uint32_t hi = 3u ^ min(a, b);
   // byte selector picking elements lo and hi out of the 8 bytes (w1:w0)
   kept = __byte_perm(w0, w1, 0x1010u + lo * 0x22u + hi * 0x2200u);
   return lo | (hi << 2);
@@ -145,6 +145,7 @@ sparsify_kernel(const __grid_constant__ SparsifyLaunch p) {
       mbar_init(&sm.empty[s], kComputeWarps);
       mbar_init(&sm.mma_done[s], 1);
     }
+    for (int v = 0; v < 2; ++v) mbar_init(&sm.vfree[v], 1);
     mbar_init(&sm.tdone, 1);
     mbar_init(&sm.drain, 1);
     sm.abort_flag = 0u;
@@ -157,25 +158,48 @@ sparsify_kernel(const __grid_constant__ SparsifyLaunch p) {
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  // finalize_kernel may begin launching; it waits for this whole grid
+  pdl_launch_dependents();
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
+    // Loads box b into stage b % kStages once box b - kStages has left it.
+    // The row threads' release of a stage also means that the kept values of
+    // that box are staged, so the same thread then issues their TMA store and,
+    // once the store has read its buffer, hands the buffer back (vfree).
     if (lane == 0) {
       tma_prefetch_desc(&p.tm_x);
       if (do_lora) tma_prefetch_desc(&p.tm_a);
+      if (do_sel) tma_prefetch_desc(&p.tm_vals);
       const uint32_t tx = kXTileBytes + (do_lora ? kATileBytes : 0u);
+      const bool store_rows = mb * 128 < p.M;  // a padding row block has metadata only
       int issued = 0;
-      if (!p.stall_test) {
-        for (int b = 0; b < nboxes; ++b) {
-          const int slot = b % kStages;
-          const uint32_t it = static_cast<uint32_t>(b / kStages);
-          if (sm.abort_flag) break;
-          // a stage is free once the row threads and the LoRA MMAs are done with it
-          if ((do_sel && !mbar_wait(&sm.empty[slot], (it & 1u) ^ 1u)) ||
-              (do_lora && !mbar_wait(&sm.mma_done[slot], (it & 1u) ^ 1u))) {
+      bool ok = !p.stall_test;
+      for (int b = 0; ok && b < nboxes + kStages; ++b) {
+        const int slot = b % kStages;
+        if (sm.abort_flag) break;
+        if (b >= kStages) {
+          const int prev = b - kStages;  // the box that last used `slot`
+          const uint32_t pph = static_cast<uint32_t>(prev / kStages) & 1u;
+          if (do_sel) {
+            if (!mbar_wait(&sm.empty[slot], pph)) {
+              set_abort(sm, p.status, kDevTimeoutEmpty);
+              break;
+            }
+            if (store_rows) {
+              tma_store_2d(&p.tm_vals, sm.vstage[prev & 1], static_cast<int32_t>((kcol0 + 64 * prev) / 2),
+                           static_cast<int32_t>(mb * 128));
+              bulk_commit();
+              bulk_wait_read_all();
+            }
+            mbar_arrive(&sm.vfree[prev & 1]);
+          }
+          if (do_lora && !mbar_wait(&sm.mma_done[slot], pph)) {
             set_abort(sm, p.status, kDevTimeoutEmpty);
             break;
           }
+        }
+        if (b < nboxes) {
           mbar_arrive_expect_tx(&sm.full[slot], tx);
           const int32_t kc = static_cast<int32_t>(kcol0 + 64 * b);
           tma_load_2d(sm.xring[slot], &p.tm_x, &sm.full[slot], kc, static_cast<int32_t>(mb * 128));
@@ -183,6 +207,7 @@ sparsify_kernel(const __grid_constant__ SparsifyLaunch p) {
           ++issued;
         }
       }
+      bulk_wait_all();  // every value tile is in global memory
       // never leave with copies in flight: wait for the last fill of each slot
       for (int b = issued - 1; b >= 0 && b >= issued - kStages; --b) {
         if (!mbar_wait(&sm.full[b % kStages], static_cast<uint32_t>(b / kStages) & 1u,
@@ -222,7 +247,6 @@ sparsify_kernel(const __grid_constant__ SparsifyLaunch p) {
     __syncwarp();
   } else if (do_sel) {
     // ------------------------------------------------------------ row threads
-    const uint32_t ct = threadIdx.x - 64;     // 0..511
     const uint32_t qt = (warp - 2) >> 2;      // which 16 columns of each tile
     const uint32_t row = 32 * (warp & 3) + lane;
     const int64_t grow = mb * 128 + row;
@@ -231,11 +255,14 @@ sparsify_kernel(const __grid_constant__ SparsifyLaunch p) {
     const uint32_t meta_hsel = (row >> 3) & 1;
     uint16_t* meta_row_blocks =
         reinterpret_cast<uint16_t*>(p.meta + static_cast<size_t>(mb) * p.kblocks * kMetaBlockBytes);
-    // where this thread's 8 kept values sit in the 64-byte-swizzled store tile
+    // where this thread's 16 bytes sit in the tile (128-byte swizzle) and its 8
+    // kept values in the 64-byte-swizzled store tile
+    const uint32_t ld_off0 = row * 128 + (((2 * qt) ^ (row & 7)) << 4);
+    const uint32_t ld_off1 = row * 128 + (((2 * qt + 1) ^ (row & 7)) << 4);
     const uint32_t vst_off = row * 64 + ((qt ^ ((row >> 1) & 3)) << 4);
-    uint64_t la2 = 0, lk2 = 0;  // (even, odd) fp32 partial sums
-    bool stop = false;
-    for (int b = 0; b < nboxes && !stop; ++b) {
+    // fp32 partial sums of |x| and |kept|, even and odd positions apart
+    float la0 = 0.f, la1 = 0.f, lk0 = 0.f, lk1 = 0.f;
+    for (int b = 0; b < nboxes; ++b) {
       const int slot = b % kStages;
       const uint32_t it = static_cast<uint32_t>(b / kStages);
       bool ok = !sm.abort_flag;
@@ -243,49 +270,40 @@ sparsify_kernel(const __grid_constant__ SparsifyLaunch p) {
         set_abort(sm, p.status, kDevTimeoutFull);
         ok = false;
       }
-      ok = __all_sync(0xffffffffu, ok);
-      if (ok) {
-        const uint8_t* tile = sm.xring[slot];
-        uint32_t kw[4];
-        uint32_t nib = 0;
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const uint32_t chunk = 2 * qt + h;
-          const uint4 v =
-              *reinterpret_cast<const uint4*>(tile + row * 128 + ((chunk ^ (row & 7)) << 4));
-          const uint32_t n0 = select_group(v.x, v.y, kw[2 * h]);
-          const uint32_t n1 = select_group(v.z, v.w, kw[2 * h + 1]);
-          nib |= (n0 | (n1 << 4)) << (8 * h);
-          la2 = add_f32x2(la2, abs_pair(v.x));
-          la2 = add_f32x2(la2, abs_pair(v.y));
-          la2 = add_f32x2(la2, abs_pair(v.z));
-          la2 = add_f32x2(la2, abs_pair(v.w));
-          lk2 = add_f32x2(lk2, abs_pair(kw[2 * h]));
-          lk2 = add_f32x2(lk2, abs_pair(kw[2 * h + 1]));
-        }
-        const int64_t kabs = kcol0 + 64 * b + 16 * qt;
-        uint16_t* blk = meta_row_blocks + static_cast<size_t>(kabs >> 7) * (kMetaBlockBytes / 2);
-        blk[meta_lane * 8 + static_cast<uint32_t>((kabs & 127) >> 5) * 2 + meta_hsel] =
-            static_cast<uint16_t>(nib);
-        *reinterpret_cast<uint4*>(sm.vstage[b & 1] + vst_off) = make_uint4(kw[0], kw[1], kw[2], kw[3]);
-        fence_proxy_async_smem();
-        // release the stage only after everything derived from it has been
-        // produced: an arrive does not wait for this warp's loads in flight
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&sm.empty[slot]);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      const uint8_t* tile = sm.xring[slot];
+      const uint4 v0 = *reinterpret_cast<const uint4*>(tile + ld_off0);
+      const uint4 v1 = *reinterpret_cast<const uint4*>(tile + ld_off1);
+      uint32_t kw[4];
+      const uint32_t n0 = select_group(v0.x, v0.y, kw[0], la0, la1);
+      const uint32_t n1 = select_group(v0.z, v0.w, kw[1], la0, la1);
+      const uint32_t n2 = select_group(v1.x, v1.y, kw[2], la0, la1);
+      const uint32_t n3 = select_group(v1.z, v1.w, kw[3], la0, la1);
+      const uint32_t nib = n0 | (n1 << 4) | (n2 << 8) | (n3 << 12);
+      add_abs_pair(lk0, lk1, kw[0]);
+      add_abs_pair(lk0, lk1, kw[1]);
+      add_abs_pair(lk0, lk1, kw[2]);
+      add_abs_pair(lk0, lk1, kw[3]);
+      const int64_t kabs = kcol0 + 64 * b + 16 * qt;
+      uint16_t* blk = meta_row_blocks + static_cast<size_t>(kabs >> 7) * (kMetaBlockBytes / 2);
+      blk[meta_lane * 8 + static_cast<uint32_t>((kabs & 127) >> 5) * 2 + meta_hsel] =
+          static_cast<uint16_t>(nib);
+      // the store of box b - 2 has read this staging buffer
+      ok = !sm.abort_flag;
+      if (ok && !mbar_wait(&sm.vfree[b & 1], static_cast<uint32_t>((b >> 1) & 1) ^ 1u)) {
+        set_abort(sm, p.status, kDevTimeoutEmpty);
+        ok = false;
       }
-      if (ct == 0) bulk_wait_read_all();  // the store of tile b-1 has read its buffer
-      stop = named_bar_red_or(kBarCompute, kComputeThreads, !ok);
-      if (!stop && ct == 0 && mb * 128 < p.M) {
-        tma_store_2d(&p.tm_vals, sm.vstage[b & 1], static_cast<int32_t>((kcol0 + 64 * b) / 2),
-                     static_cast<int32_t>(mb * 128));
-        bulk_commit();
-      }
+      if (!__all_sync(0xffffffffu, ok)) break;
+      *reinterpret_cast<uint4*>(sm.vstage[b & 1] + vst_off) = make_uint4(kw[0], kw[1], kw[2], kw[3]);
+      fence_proxy_async_smem();
+      // release the stage only after everything derived from it has been
+      // produced: an arrive does not wait for this warp's loads in flight
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.empty[slot]);
     }
-    const float my_la = __fadd_rn(__uint_as_float(static_cast<uint32_t>(la2)),
-                                  __uint_as_float(static_cast<uint32_t>(la2 >> 32)));
-    const float my_lk = __fadd_rn(__uint_as_float(static_cast<uint32_t>(lk2)),
-                                  __uint_as_float(static_cast<uint32_t>(lk2 >> 32)));
+    const float my_la = __fadd_rn(la0, la1);
+    const float my_lk = __fadd_rn(lk0, lk1);
     if (qt > 0) sm.quarter[qt - 1][row] = make_float2(my_la, my_lk);
     named_bar_sync(kBarCompute, kComputeThreads);
     if (qt == 0 && grow < p.M) {
@@ -298,7 +316,6 @@ sparsify_kernel(const __grid_constant__ SparsifyLaunch p) {
       }
       p.lpart[static_cast<size_t>(j) * p.M + grow] = make_float2(a, k);
     }
-    if (ct == 0) bulk_wait_all();  // every value tile is in global memory
   }
 
   // ---- T partial of this K range: TMEM -> registers -> global (fp32)
@@ -336,27 +353,44 @@ __global__ void __launch_bounds__(256)
 finalize_kernel(const float2* __restrict__ lpart, const float* __restrict__ tpart, int64_t M,
                 int C, int do_scale, int do_lora, int divide, float* __restrict__ row_scale,
                 __nv_bfloat16* __restrict__ t_out) {
+  pdl_launch_dependents();
+  pdl_wait();  // the partials of sparsify_kernel
   const int64_t row = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
   const uint32_t lane = threadIdx.x & 31u;
   if (row >= M) return;
   float s = 1.f;
+  // all C partials are loaded before any is added (the loads overlap), then
+  // summed in the fixed order j = 0, 1, ...
   if (do_scale) {
+    float2 v[kMaxSplit];
+#pragma unroll
+    for (int j = 0; j < kMaxSplit; ++j)
+      if (j < C) v[j] = __ldcg(lpart + static_cast<size_t>(j) * M + row);
     float la = 0.f, lk = 0.f;
-    for (int j = 0; j < C; ++j) {
-      const float2 v = __ldcg(lpart + static_cast<size_t>(j) * M + row);
-      la = __fadd_rn(la, v.x);
-      lk = __fadd_rn(lk, v.y);
+#pragma unroll
+    for (int j = 0; j < kMaxSplit; ++j) {
+      if (j < C) {
+        la = __fadd_rn(la, v[j].x);
+        lk = __fadd_rn(lk, v[j].y);
+      }
     }
     s = (lk == 0.f) ? 1.f : __fdiv_rn(la, lk);
     if (lane == 0) row_scale[row] = s;
   }
   if (do_lora) {
-    float a0 = 0.f, a1 = 0.f;  // columns 2*lane, 2*lane+1
-    for (int j = 0; j < C; ++j) {
-      const float2 v = __ldcg(reinterpret_cast<const float2*>(
-          tpart + (static_cast<size_t>(j) * M + row) * kLoraRank) + lane);
-      a0 = __fadd_rn(a0, v.x);
-      a1 = __fadd_rn(a1, v.y);
+    float2 v[kMaxSplit];  // columns 2*lane, 2*lane+1 of each partial
+#pragma unroll
+    for (int j = 0; j < kMaxSplit; ++j)
+      if (j < C)
+        v[j] = __ldcg(reinterpret_cast<const float2*>(
+                          tpart + (static_cast<size_t>(j) * M + row) * kLoraRank) + lane);
+    float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+    for (int j = 0; j < kMaxSplit; ++j) {
+      if (j < C) {
+        a0 = __fadd_rn(a0, v[j].x);
+        a1 = __fadd_rn(a1, v[j].y);
+      }
     }
     if (divide) {
       a0 = __fdiv_rn(a0, s);
@@ -371,6 +405,7 @@ finalize_kernel(const float2* __restrict__ lpart, const float* __restrict__ tpar
 __global__ void __launch_bounds__(256)
 rescale_kernel(uint4* __restrict__ vals, const float* __restrict__ row_scale, int64_t M,
                int64_t K) {
+  pdl_wait();  // s from finalize_kernel, values from sparsify_kernel
   const int64_t per_row = K / 16;  // uint4 per row (K/2 bf16 = K bytes)
   const int64_t total = M * per_row;
   for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
@@ -420,16 +455,17 @@ cudaError_t launch_sparsify(const SparsifyLaunch& p, cudaStream_t stream) {
   const bool do_lora = (p.mode & kModeLora) != 0;
   const bool scaled = (p.mode & kModeScaled) != 0;
   const unsigned fin_blocks = static_cast<unsigned>((p.M + 7) / 8);
-  finalize_kernel<<<fin_blocks, 256, 0, stream>>>(p.lpart, p.tpart, p.M, p.split, do_sel ? 1 : 0,
-                                                  do_lora ? 1 : 0, (do_sel && !scaled) ? 1 : 0,
-                                                  p.row_scale,
-                                                  static_cast<__nv_bfloat16*>(p.t_out));
-  e = cudaGetLastError();
+  e = launch_after_previous(finalize_kernel, dim3(fin_blocks), dim3(256), 0, stream,
+                            static_cast<const float2*>(p.lpart), static_cast<const float*>(p.tpart),
+                            p.M, p.split, do_sel ? 1 : 0, do_lora ? 1 : 0,
+                            (do_sel && !scaled) ? 1 : 0, p.row_scale,
+                            static_cast<__nv_bfloat16*>(p.t_out));
   if (e != cudaSuccess || !(do_sel && scaled)) return e;
   const int64_t n16 = p.M * (p.K / 16);
   const unsigned rb = static_cast<unsigned>(std::min<int64_t>((n16 + 255) / 256, 4096));
-  rescale_kernel<<<rb, 256, 0, stream>>>(static_cast<uint4*>(p.vals), p.row_scale, p.M, p.K);
-  return cudaGetLastError();
+  return launch_after_previous(rescale_kernel, dim3(rb), dim3(256), 0, stream,
+                               static_cast<uint4*>(p.vals), static_cast<const float*>(p.row_scale),
+                               p.M, p.K);
 }
 
 }  // namespace lynx

@@ -197,6 +197,8 @@ LYNX_API int lynx_meta_canonical_to_hw(const uint8_t* canonical, uint8_t* hw, in
  * lynx_linear records it on its stream between the sparsify pass and the GEMM,
  * so a caller can time the two kernels of one call separately with events
  * recorded before and after the call.  NULL (the default) turns it off.
+ * While it is set, the GEMM no longer starts (programmatic launch) during the
+ * tail of the sparsify pass, so a call takes slightly longer.
  * Process-wide; returns the previous event. */
 LYNX_API void* lynx_profile_set_split_event(void* event);
 
