@@ -1,0 +1,75 @@
+"""The block sweep replayed from a CUDA graph: every layer's Y from the graph
+equals the eagerly launched sequence bit for bit, and sampled rows of one
+layer of each kind (a dense, skip_sparsify block among them) match the oracle
+within the layer's tolerance."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from activation_sparse_gemm_lynx_b200 import lynx, workloads
+from activation_sparse_gemm_lynx_b200.sweep import LinearSweep
+
+import helpers
+
+pytestmark = pytest.mark.gpu
+
+
+def host(t):
+    return t.detach().contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+
+
+@pytest.fixture(scope="module")
+def sweep_and_plan():
+    assert torch.cuda.is_available(), "these tests need a GPU"
+    torch.cuda.set_device(0)
+    lynx.library()
+    lynx.lynx_check_error()
+    # the sweep's layer shapes and skip pattern at a reduced token count
+    # (384 rows: one and a half CTA-pair row blocks)
+    plan = workloads.sweep_plan(M=384)
+    layers = []
+    for (_b, _n, M, K, N, kind, skip, seed) in plan:
+        inp = workloads.make_linear_inputs(M, K, N, seed=seed, x_kind=kind)
+        inp["skip"] = skip
+        layers.append(inp)
+    return LinearSweep(layers, device="cuda:0"), plan, layers
+
+
+def test_graph_replay_equals_eager_pass(sweep_and_plan):
+    sweep, plan, _ = sweep_and_plan
+    sweep.run()
+    torch.cuda.synchronize()
+    eager = [t["Y"].clone() for t in sweep.layers]
+    for t in sweep.layers:
+        t["Y"].zero_()
+    sweep.capture()
+    sweep.replay()
+    sweep.replay()  # twice: the shared workspace is reused in place
+    torch.cuda.synchronize()
+    st, code = lynx.lynx_check_error()
+    assert st == lynx.LYNX_OK, (st, code)
+    for i, (t, e) in enumerate(zip(sweep.layers, eager)):
+        assert torch.equal(t["Y"].view(torch.int16), e.view(torch.int16)), plan[i][:2]
+
+
+def test_graph_layers_match_oracle(sweep_and_plan):
+    sweep, plan, layers = sweep_and_plan
+    if sweep.graph is None:
+        sweep.run()
+        sweep.capture()
+    sweep.replay()
+    torch.cuda.synchronize()
+    skipped = {b for (b, _n, *_r, skip, _s) in plan if skip}
+    assert len(skipped) == 2
+    first_dense = min(skipped)
+    picked = [i for i, p in enumerate(plan) if p[0] == 0] + \
+             [i for i, p in enumerate(plan) if p[0] == first_dense]
+    rows = np.array([0, 1, 127, 128, 255, 256, 383])
+    for i in picked:
+        inp = layers[i]
+        y = helpers.f32(host(sweep.layers[i]["Y"])).astype(np.float64)[rows]
+        y_ref, _, sx = oracle.linear(inp["X"][rows], inp["W"], inp["bias"], inp["A"], inp["B"],
+                                     skip=inp["skip"], want_sx=True)
+        worst, fro = helpers.y_tolerance_check(y, y_ref, sx, helpers.f32(inp["W"]).astype(np.float64))
+        assert worst <= 1.0 and fro <= 5e-3, (plan[i][:2], worst, fro)
