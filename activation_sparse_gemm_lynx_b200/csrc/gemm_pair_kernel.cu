@@ -23,6 +23,12 @@
 //   warps 2-9   epilogue on the CTA's own 128 accumulator rows: s * acc + bias
 //               -> bf16 -> global; releases the accumulator by arriving on the
 //               leader's "acc_empty" barrier.
+//   warp 10     in the leader CTA: waits for each filled stage ("full") and
+//               hands it to the MMA issuer through a named barrier.  A
+//               shared-memory barrier poll in the issuing warp itself costs the
+//               tensor pipe about a fifth of its rate when the operands change
+//               from stage to stage; a hardware barrier between two warps does
+//               not.
 #include <cuda_bf16.h>
 
 #include "lynx_internal.h"
@@ -32,7 +38,10 @@ namespace lynx {
 
 namespace {
 
-constexpr int kThreads = 320;
+constexpr int kThreads = 352;
+constexpr uint32_t kHelperWarp = 10;
+constexpr uint32_t kBarStage0 = 3;  // named barriers 3 .. 3 + stages - 1: stage hand-off
+constexpr uint32_t kHandoffThreads = 64;  // the MMA warp and the helper warp
 constexpr uint32_t kTmemCols = 512;
 constexpr int kEslots = 4;
 constexpr uint32_t kBarEpilogue = 2;
@@ -57,6 +66,7 @@ struct PairCfg {
   static constexpr uint32_t kLoraABytes = 128u * 64u;  // T: own 128 rows x 32
   static constexpr uint32_t kLoraBBytes = 128u * 64u;  // B: own 128 rows x 32
   static_assert(kStages >= 4, "pipeline too shallow");
+  static_assert(kBarStage0 + kStages <= 16, "named barriers");
 };
 
 template <bool SPARSE>
@@ -201,31 +211,23 @@ lynx_gemm_pair_kernel(const __grid_constant__ GemmLaunch p) {
       const uint32_t idesc_dense = make_idesc_bf16(256, 256, false);
       uint32_t g = 0, eslot = 0;
       int acc_count = 0;
-      bool ok = true;
-      for (int tile = cluster_id; ok && tile < ntiles; tile += nclusters, ++acc_count) {
-        bool got = !sm.abort_flag && mbar_wait(&sm.acc_empty, (static_cast<uint32_t>(acc_count) & 1u) ^ 1u);
-        got = __all_sync(0xffffffffu, got);
-        if (!got) {
-          if (!sm.abort_flag && lane == 0) {
-            record_error(p.status, kDevTimeoutAccum);
-            sm.abort_flag = 1u;
-          }
-          break;
+      bool stop = false;
+      for (int tile = cluster_id; !stop && tile < ntiles; tile += nclusters, ++acc_count) {
+        bool err = sm.abort_flag || !mbar_wait(&sm.acc_empty, (static_cast<uint32_t>(acc_count) & 1u) ^ 1u);
+        err = __any_sync(0xffffffffu, err);
+        if (err && lane == 0 && !sm.abort_flag) {
+          record_error(p.status, kDevTimeoutAccum);
+          sm.abort_flag = 1u;
         }
         tc_fence_after();
         const uint32_t d_tmem = sm.tmem_base;
         uint32_t accumulate = 0;
         for (int kit = 0; kit < steps; ++kit, ++g) {
           const uint32_t slot = g % C::kStages;
-          const uint32_t ph = (g / C::kStages) & 1u;
-          bool ready = !sm.abort_flag && mbar_wait(&sm.full[slot], ph);
-          ready = __all_sync(0xffffffffu, ready);
-          if (!ready) {
-            if (!sm.abort_flag && lane == 0) {
-              record_error(p.status, kDevTimeoutFull);
-              sm.abort_flag = 1u;
-            }
-            ok = false;
+          // the helper warp says when stage g has landed; both warps leave
+          // together (same barrier, same reduced flag) once either saw an error
+          if (named_bar_red_or(kBarStage0 + slot, kHandoffThreads, err || sm.abort_flag)) {
+            stop = true;
             break;
           }
           tc_fence_after();
@@ -271,13 +273,38 @@ lynx_gemm_pair_kernel(const __grid_constant__ GemmLaunch p) {
           if (elect_one()) tc_commit_pair_mc(&sm.empty[slot], kPairMask);
           __syncwarp();
         }
-        if (!ok) break;
+        if (stop) break;
         if (elect_one()) tc_commit_pair_mc(&sm.acc_full, kPairMask);
         __syncwarp();
       }
       if (elect_one()) tc_commit_pair_mc(&sm.drain, 0x1);
       __syncwarp();
       if (!mbar_wait(&sm.drain, 0) && lane == 0) record_error(p.status, kDevTimeoutDrain);
+    }
+    __syncwarp();
+  } else if (warp == kHelperWarp) {
+    // ------------------------------------------------------------ stage hand-off (leader)
+    // Walks the same (tile, stage) sequence as the MMA issuer: one barrier
+    // round per stage, in the same order, so every round has both warps.
+    if (leader) {
+      uint32_t g = 0;
+      bool stop = false;
+      for (int tile = cluster_id; !stop && tile < ntiles; tile += nclusters) {
+        for (int kit = 0; kit < steps; ++kit, ++g) {
+          const uint32_t slot = g % C::kStages;
+          const uint32_t ph = (g / C::kStages) & 1u;
+          bool ok = !sm.abort_flag && mbar_wait(&sm.full[slot], ph);
+          ok = __all_sync(0xffffffffu, ok);
+          if (!ok && lane == 0 && !sm.abort_flag) {
+            record_error(p.status, kDevTimeoutFull);
+            sm.abort_flag = 1u;
+          }
+          if (named_bar_red_or(kBarStage0 + slot, kHandoffThreads, !ok)) {
+            stop = true;
+            break;
+          }
+        }
+      }
     }
     __syncwarp();
   } else {
