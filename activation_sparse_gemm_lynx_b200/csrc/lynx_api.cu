@@ -172,9 +172,9 @@ lynx_status run_sparsify(DeviceState* ds, const void* X, const void* A, int64_t 
 }
 
 // CTA pairs (256 x 256 tiles) unless the problem is too small to feed them; the
-// sparse pair kernel steps K by 128
-bool use_pair_kernel(int64_t M, int64_t N, int64_t K, bool sparse) {
-  return M > 128 && N >= 256 && (!sparse || K % 128 == 0);
+// pair kernel steps K by 128 on both paths
+bool use_pair_kernel(int64_t M, int64_t N, int64_t K) {
+  return M > 128 && N >= 256 && K % 128 == 0;
 }
 
 lynx_status run_gemm(DeviceState* ds, const void* a_src, bool sparse, const void* meta,
@@ -182,7 +182,7 @@ lynx_status run_gemm(DeviceState* ds, const void* a_src, bool sparse, const void
                      const void* B, int64_t M, int64_t N, int64_t K, void* Y, cudaStream_t stream) {
   GemmLaunch p;
   std::memset(&p, 0, sizeof(p));
-  const bool pair = use_pair_kernel(M, N, K, sparse);
+  const bool pair = use_pair_kernel(M, N, K);
   const int bn = pair ? 256 : gemm_bn(N);
   const uint32_t b_rows = pair ? 128u : static_cast<uint32_t>(bn);  // W rows one CTA loads
   if (sparse) {
