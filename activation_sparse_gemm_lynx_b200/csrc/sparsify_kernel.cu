@@ -158,6 +158,10 @@ sparsify_kernel(const __grid_constant__ SparsifyLaunch p) {
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  // the prologue above may overlap the previous kernel on the stream; X (its
+  // output, possibly) is read and this call's outputs (possibly still read by
+  // it) are written only from here on
+  pdl_wait();
   // finalize_kernel may begin launching; it waits for this whole grid
   pdl_launch_dependents();
 
@@ -262,11 +266,15 @@ sparsify_kernel(const __grid_constant__ SparsifyLaunch p) {
     const uint32_t vst_off = row * 64 + ((qt ^ ((row >> 1) & 3)) << 4);
     // fp32 partial sums of |x| and |kept|, even and odd positions apart
     float la0 = 0.f, la1 = 0.f, lk0 = 0.f, lk1 = 0.f;
-    for (int b = 0; b < nboxes; ++b) {
-      const int slot = b % kStages;
-      const uint32_t it = static_cast<uint32_t>(b / kStages);
+    // this thread's metadata field of box b: block (kabs >> 7) of the row
+    // block, 16-bit word lane*8 + ((kabs >> 5) & 3)*2 + hsel, kabs = its first
+    // dense column (32-bit: K < 2^30)
+    const uint32_t meta_lane_off = meta_lane * 8 + meta_hsel;
+    uint32_t kabs = static_cast<uint32_t>(kcol0) + 16 * qt;
+    uint32_t slot = 0, phase = 0;
+    for (int b = 0; b < nboxes; ++b, kabs += 64) {
       bool ok = !sm.abort_flag;
-      if (ok && !mbar_wait(&sm.full[slot], it & 1u)) {
+      if (ok && !mbar_wait(&sm.full[slot], phase)) {
         set_abort(sm, p.status, kDevTimeoutFull);
         ok = false;
       }
@@ -284,13 +292,10 @@ sparsify_kernel(const __grid_constant__ SparsifyLaunch p) {
       add_abs_pair(lk0, lk1, kw[1]);
       add_abs_pair(lk0, lk1, kw[2]);
       add_abs_pair(lk0, lk1, kw[3]);
-      const int64_t kabs = kcol0 + 64 * b + 16 * qt;
-      uint16_t* blk = meta_row_blocks + static_cast<size_t>(kabs >> 7) * (kMetaBlockBytes / 2);
-      blk[meta_lane * 8 + static_cast<uint32_t>((kabs & 127) >> 5) * 2 + meta_hsel] =
+      meta_row_blocks[((kabs >> 7) << 10) + meta_lane_off + (((kabs >> 5) & 3u) << 1)] =
           static_cast<uint16_t>(nib);
       // the store of box b - 2 has read this staging buffer
-      ok = !sm.abort_flag;
-      if (ok && !mbar_wait(&sm.vfree[b & 1], static_cast<uint32_t>((b >> 1) & 1) ^ 1u)) {
+      if (!mbar_wait(&sm.vfree[b & 1], static_cast<uint32_t>((b >> 1) & 1) ^ 1u)) {
         set_abort(sm, p.status, kDevTimeoutEmpty);
         ok = false;
       }
@@ -301,6 +306,10 @@ sparsify_kernel(const __grid_constant__ SparsifyLaunch p) {
       // produced: an arrive does not wait for this warp's loads in flight
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.empty[slot]);
+      if (++slot == kStages) {
+        slot = 0;
+        phase ^= 1u;
+      }
     }
     const float my_la = __fadd_rn(la0, la1);
     const float my_lk = __fadd_rn(lk0, lk1);
@@ -448,8 +457,7 @@ cudaError_t launch_sparsify(const SparsifyLaunch& p, cudaStream_t stream) {
   // metadata row blocks come in pairs: the block past M (if any) gets the
   // pattern of all-zero rows, so a CTA pair of the GEMM never reads garbage
   const dim3 grid(static_cast<unsigned>(p.split), static_cast<unsigned>(meta_row_blocks(p.M)), 1);
-  sparsify_kernel<<<grid, kThreads, smem, stream>>>(p);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_after_previous(sparsify_kernel, grid, dim3(kThreads), smem, stream, p);
   if (e != cudaSuccess) return e;
   const bool do_sel = (p.mode & kModeSelect) != 0;
   const bool do_lora = (p.mode & kModeLora) != 0;
