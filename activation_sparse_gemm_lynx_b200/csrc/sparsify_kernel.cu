@@ -151,6 +151,23 @@ sparsify_kernel(const __grid_constant__ SparsifyLaunch p) {
     sm.abort_flag = 0u;
     fence_mbar_init();
   }
+  // The first stages' loads leave before the rest of the prologue (TMEM
+  // allocation, the block barrier): the first box is the one whose latency
+  // nothing else hides.  They wait for the previous kernel like every access
+  // to X below.
+  const int preissued = (nboxes < kStages) ? nboxes : kStages;
+  if (threadIdx.x == 0 && !p.stall_test) {
+    tma_prefetch_desc(&p.tm_x);
+    if (do_lora) tma_prefetch_desc(&p.tm_a);
+    pdl_wait();
+    const uint32_t tx = kXTileBytes + (do_lora ? kATileBytes : 0u);
+    for (int b = 0; b < preissued; ++b) {
+      mbar_arrive_expect_tx(&sm.full[b], tx);
+      const int32_t kc = static_cast<int32_t>(kcol0 + 64 * b);
+      tma_load_2d(sm.xring[b], &p.tm_x, &sm.full[b], kc, static_cast<int32_t>(mb * 128));
+      if (do_lora) tma_load_2d(sm.aring[b], &p.tm_a, &sm.full[b], kc, 0);
+    }
+  }
   if (warp == 1 && do_lora) {
     tmem_alloc(&sm.tmem_base, kTmemCols);
     tmem_relinquish();
@@ -172,13 +189,11 @@ sparsify_kernel(const __grid_constant__ SparsifyLaunch p) {
     // that box are staged, so the same thread then issues their TMA store and,
     // once the store has read its buffer, hands the buffer back (vfree).
     if (lane == 0) {
-      tma_prefetch_desc(&p.tm_x);
-      if (do_lora) tma_prefetch_desc(&p.tm_a);
       if (do_sel) tma_prefetch_desc(&p.tm_vals);
       const uint32_t tx = kXTileBytes + (do_lora ? kATileBytes : 0u);
       const bool store_rows = mb * 128 < p.M;  // a padding row block has metadata only
-      int issued = 0;
       bool ok = !p.stall_test;
+      int issued = ok ? preissued : 0;
       for (int b = 0; ok && b < nboxes + kStages; ++b) {
         const int slot = b % kStages;
         if (sm.abort_flag) break;
@@ -203,7 +218,7 @@ sparsify_kernel(const __grid_constant__ SparsifyLaunch p) {
             break;
           }
         }
-        if (b < nboxes) {
+        if (b >= preissued && b < nboxes) {
           mbar_arrive_expect_tx(&sm.full[slot], tx);
           const int32_t kc = static_cast<int32_t>(kcol0 + 64 * b);
           tma_load_2d(sm.xring[slot], &p.tm_x, &sm.full[slot], kc, static_cast<int32_t>(mb * 128));
