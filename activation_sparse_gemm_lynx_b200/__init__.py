@@ -18,6 +18,8 @@ from .lynx import (  # noqa: F401
     lynx_debug_set_stall,
     lynx_linear,
     lynx_linear_dense,
+    lynx_linear_host,
+    lynx_linear_host_workspace_bytes,
     lynx_lora_rank,
     lynx_meta_bytes,
     lynx_meta_canonical_to_hw,

@@ -39,6 +39,54 @@ struct DeviceState {
 };
 DeviceState g_dev[kMaxDevices];
 
+// Streams and events of lynx_linear_host, made once per device: copies in and
+// copies out run on their own streams so that they overlap each other (the link
+// is full duplex) and the kernels on the caller's stream.
+constexpr int kHostMaxChunks = 8;
+struct HostPipe {
+  std::once_flag once;
+  std::mutex enqueue;  // one call's enqueue sequence at a time (events are reused)
+  cudaStream_t in = nullptr, out = nullptr;
+  cudaEvent_t start = nullptr, out_done = nullptr;
+  cudaEvent_t in_done[kHostMaxChunks] = {};
+  cudaEvent_t comp_done[kHostMaxChunks] = {};
+  cudaError_t err = cudaSuccess;
+};
+HostPipe g_host[kMaxDevices];
+
+HostPipe* host_pipe() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  HostPipe& h = g_host[dev];
+  std::call_once(h.once, [&h]() {
+    auto ok = [&h](cudaError_t e) {
+      if (h.err == cudaSuccess) h.err = e;
+      return h.err == cudaSuccess;
+    };
+    ok(cudaStreamCreateWithFlags(&h.in, cudaStreamNonBlocking));
+    ok(cudaStreamCreateWithFlags(&h.out, cudaStreamNonBlocking));
+    ok(cudaEventCreateWithFlags(&h.start, cudaEventDisableTiming));
+    ok(cudaEventCreateWithFlags(&h.out_done, cudaEventDisableTiming));
+    for (int i = 0; i < kHostMaxChunks; ++i) {
+      ok(cudaEventCreateWithFlags(&h.in_done[i], cudaEventDisableTiming));
+      ok(cudaEventCreateWithFlags(&h.comp_done[i], cudaEventDisableTiming));
+    }
+  });
+  return h.err == cudaSuccess ? &h : nullptr;
+}
+
+// Row chunks of lynx_linear_host: up to kHostMaxChunks, each a multiple of 256
+// rows (the GEMM's CTA-pair row block) and, but for a single chunk, at least
+// 512.  The copy of the last chunk back to the host is the part that nothing
+// overlaps, so more, smaller chunks shorten it; the layer on a chunk runs well
+// under the time of its copies.
+int64_t host_chunk_rows(int64_t M) {
+  int64_t n = M / 512;
+  n = n < 1 ? 1 : (n > kHostMaxChunks ? kHostMaxChunks : n);
+  const int64_t rows = (M + n - 1) / n;
+  return ((rows + 255) / 256) * 256;
+}
+
 void resolve_encode() {
   void* fn = nullptr;
   cudaDriverEntryPointQueryResult q;
@@ -404,6 +452,64 @@ int lynx_linear(const void* X, const void* W, const void* bias, const void* A, c
   if (void* ev = g_split_event.load())
     if (cudaEventRecord(static_cast<cudaEvent_t>(ev), s) != cudaSuccess) return LYNX_ERR_CUDA;
   return run_gemm(ds, X, false, nullptr, nullptr, t_buf, W, bias, B, M, N, K, Y, s);
+}
+
+size_t lynx_linear_host_workspace_bytes(int64_t M, int64_t N, int64_t K, int64_t r) {
+  if (M <= 0 || N <= 0 || K <= 0) return 0;
+  const size_t x = align256(static_cast<size_t>(M) * static_cast<size_t>(K) * 2);
+  const size_t y = align256(static_cast<size_t>(M) * static_cast<size_t>(N) * 2);
+  return x + y + lynx_workspace_bytes(host_chunk_rows(M), N, K, r);
+}
+
+int lynx_linear_host(const void* X_host, const void* W, const void* bias, const void* A, const void* B,
+                     int64_t M, int64_t N, int64_t K, int64_t r, int skip_sparsify, void* Y_host,
+                     void* workspace, size_t workspace_bytes, void* stream) {
+  if (X_host == nullptr || W == nullptr || Y_host == nullptr || workspace == nullptr)
+    return LYNX_ERR_INVALID_ARG;
+  lynx_status st = check_lora(A, B, r);
+  if (st != LYNX_OK) return st;
+  st = check_shape(M, N, K);
+  if (st != LYNX_OK) return st;
+  if (!aligned16(workspace)) return LYNX_ERR_MISALIGNED;
+  if (workspace_bytes < lynx_linear_host_workspace_bytes(M, N, K, r)) return LYNX_ERR_WORKSPACE_TOO_SMALL;
+  HostPipe* hp = host_pipe();
+  if (hp == nullptr) return LYNX_ERR_CUDA;
+  std::lock_guard<std::mutex> guard(hp->enqueue);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  uint8_t* x_dev = ws;
+  uint8_t* y_dev = ws + align256(static_cast<size_t>(M) * static_cast<size_t>(K) * 2);
+  uint8_t* layer_ws = y_dev + align256(static_cast<size_t>(M) * static_cast<size_t>(N) * 2);
+  const int64_t rows = host_chunk_rows(M);
+  const size_t layer_bytes = lynx_workspace_bytes(rows, N, K, r);
+  const size_t xrow = static_cast<size_t>(K) * 2, yrow = static_cast<size_t>(N) * 2;
+  // the copies start after the work already on the caller's stream (which may
+  // still use the workspace)
+  if (cudaEventRecord(hp->start, s) != cudaSuccess || cudaStreamWaitEvent(hp->in, hp->start, 0) != cudaSuccess ||
+      cudaStreamWaitEvent(hp->out, hp->start, 0) != cudaSuccess)
+    return LYNX_ERR_CUDA;
+  int chunk = 0;
+  for (int64_t m0 = 0; m0 < M; m0 += rows, ++chunk) {
+    const int64_t mc = (M - m0 < rows) ? (M - m0) : rows;
+    const size_t off_x = static_cast<size_t>(m0) * xrow, off_y = static_cast<size_t>(m0) * yrow;
+    if (cudaMemcpyAsync(x_dev + off_x, static_cast<const uint8_t*>(X_host) + off_x,
+                        static_cast<size_t>(mc) * xrow, cudaMemcpyHostToDevice, hp->in) != cudaSuccess ||
+        cudaEventRecord(hp->in_done[chunk], hp->in) != cudaSuccess ||
+        cudaStreamWaitEvent(s, hp->in_done[chunk], 0) != cudaSuccess)
+      return LYNX_ERR_CUDA;
+    st = static_cast<lynx_status>(lynx_linear(x_dev + off_x, W, bias, A, B, mc, N, K, r, skip_sparsify,
+                                              y_dev + off_y, layer_ws, layer_bytes, s));
+    if (st != LYNX_OK) return st;
+    if (cudaEventRecord(hp->comp_done[chunk], s) != cudaSuccess ||
+        cudaStreamWaitEvent(hp->out, hp->comp_done[chunk], 0) != cudaSuccess ||
+        cudaMemcpyAsync(static_cast<uint8_t*>(Y_host) + off_y, y_dev + off_y, static_cast<size_t>(mc) * yrow,
+                        cudaMemcpyDeviceToHost, hp->out) != cudaSuccess)
+      return LYNX_ERR_CUDA;
+  }
+  // later work on the caller's stream (and a synchronize of it) sees Y in host memory
+  if (cudaEventRecord(hp->out_done, hp->out) != cudaSuccess || cudaStreamWaitEvent(s, hp->out_done, 0) != cudaSuccess)
+    return LYNX_ERR_CUDA;
+  return LYNX_OK;
 }
 
 int lynx_linear_dense(const void* X, const void* W, const void* bias, const void* A,

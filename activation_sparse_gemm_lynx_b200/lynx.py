@@ -57,6 +57,8 @@ def library():
             "lynx_sparsify_noalloc_max_rows": ([], i64),
             "lynx_linear": ([p, p, p, p, p, i64, i64, i64, i64, i32, p, p, sz, p], i32),
             "lynx_linear_dense": ([p, p, p, p, p, i64, i64, i64, i64, p, p, sz, p], i32),
+            "lynx_linear_host_workspace_bytes": ([i64, i64, i64, i64], sz),
+            "lynx_linear_host": ([p, p, p, p, p, i64, i64, i64, i64, i32, p, p, sz, p], i32),
             "lynx_sparse_gemm": ([p, p, p, p, p, p, i64, i64, i64, i64, p, p], i32),
             "lynx_check_error": ([p, p], i32),
             "lynx_meta_hw_to_canonical": ([p, p, i64, i64], i32),
@@ -231,6 +233,50 @@ def lynx_linear(X, W, bias=None, A=None, B=None, skip_sparsify=False, Y=None, wo
                                workspace.numel(), _stream(stream))
     _check(st, "lynx_linear")
     return Y
+
+
+def lynx_linear_host_workspace_bytes(M, N, K, r=64):
+    return library().lynx_linear_host_workspace_bytes(M, N, K, r)
+
+
+def lynx_linear_host(X_host, W, bias=None, A=None, B=None, skip_sparsify=False, Y_host=None,
+                     workspace=None, stream=None):
+    """The layer on host activations: X_host [M,K] and Y_host [M,N] are CPU bf16
+    tensors (pinned for asynchronous copies); W, bias, A, B are CUDA tensors.
+    Returns Y_host, complete once `stream` (default: the current stream) has
+    reached this point."""
+    import torch
+
+    if X_host is None or X_host.is_cuda or X_host.dtype != torch.bfloat16 or not X_host.is_contiguous():
+        raise ValueError("X_host must be a contiguous bf16 CPU tensor")
+    _need(W, "W", torch.bfloat16)
+    M, K = X_host.shape
+    N = W.shape[0]
+    if W.shape[1] != K:
+        raise ValueError("W must be [N,K]")
+    if bias is not None:
+        _need(bias, "bias", torch.bfloat16, (N,))
+    if (A is None) != (B is None):
+        raise ValueError("A and B must both be given or both be None")
+    r = 0
+    if A is not None:
+        r = A.shape[0]
+        _need(A, "A", torch.bfloat16, (r, K))
+        _need(B, "B", torch.bfloat16, (N, r))
+    if Y_host is None:
+        Y_host = torch.empty((M, N), dtype=torch.bfloat16).pin_memory()
+    if Y_host.is_cuda or Y_host.dtype != torch.bfloat16 or tuple(Y_host.shape) != (M, N) or \
+            not Y_host.is_contiguous():
+        raise ValueError("Y_host must be a contiguous bf16 CPU tensor of shape [M,N]")
+    need = lynx_linear_host_workspace_bytes(M, N, K, r if r else 64)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=W.device)
+    _need(workspace, "workspace", torch.uint8)
+    st = library().lynx_linear_host(_ptr(X_host), _ptr(W), _ptr(bias), _ptr(A), _ptr(B), M, N, K, r,
+                                    1 if skip_sparsify else 0, _ptr(Y_host), _ptr(workspace),
+                                    workspace.numel(), _stream(stream))
+    _check(st, "lynx_linear_host")
+    return Y_host
 
 
 def lynx_linear_dense(X, W, bias=None, A=None, B=None, Y=None, workspace=None, stream=None):

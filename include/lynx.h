@@ -162,6 +162,29 @@ LYNX_API int lynx_linear(const void* X, const void* W, const void* bias, const v
                 int64_t M, int64_t N, int64_t K, int64_t r, int skip_sparsify, void* Y,
                 void* workspace, size_t workspace_bytes, void* stream);
 
+/* ---- the layer on host-memory activations ------------------------------ */
+
+/* Bytes of the device workspace lynx_linear_host needs: device copies of X and
+ * Y plus the layer workspace of one row chunk. */
+LYNX_API size_t lynx_linear_host_workspace_bytes(int64_t M, int64_t N, int64_t K, int64_t r);
+
+/* lynx_linear with X [M,K] and Y [M,N] in host memory (page-locked for the copies
+ * to run asynchronously); W, bias, A, B stay device pointers.  The rows are
+ * processed in up to 8 chunks (multiples of 256 rows): the copy of chunk i+1 into
+ * the device, the layer on chunk i and the copy of chunk i-1 back to the host run
+ * at the same time, the two copy directions on internal streams of the library.
+ * The work is ordered after everything already enqueued on `stream`, and
+ * anything enqueued on `stream` afterwards (a synchronize included) sees Y
+ * complete in host memory.  Results equal lynx_linear's, row for row.
+ *   workspace: device buffer of workspace_bytes >= lynx_linear_host_workspace_bytes.
+ *   Errors as lynx_linear.  The first call on a device creates its two streams
+ *   and its events.  Enqueues from several host threads are serialised inside
+ *   the call; each call needs its own workspace and Y. */
+LYNX_API int lynx_linear_host(const void* X_host, const void* W, const void* bias, const void* A,
+                              const void* B, int64_t M, int64_t N, int64_t K, int64_t r,
+                              int skip_sparsify, void* Y_host, void* workspace,
+                              size_t workspace_bytes, void* stream);
+
 /* The dense path of a layer that selective layer skipping leaves dense
  * (qingkeai.online article section 03.3): Y = X W^T + bias + (X A^T) B^T.
  * Same arguments and workspace as lynx_linear. */

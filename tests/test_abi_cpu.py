@@ -95,6 +95,24 @@ def test_sparsify_argument_errors(lib):
         lynx.LYNX_ERR_WORKSPACE_TOO_SMALL
 
 
+def test_linear_host_argument_errors(lib):
+    f = lib.lynx_linear_host
+    need = lynx.lynx_linear_host_workspace_bytes(256, 512, 512, 64)
+    assert need >= 2 * 256 * 512 * 2 + lynx.lynx_workspace_bytes(256, 512, 512, 64)
+
+    def call(X=P, W=P, Y=P, ws=P, ws_bytes=need, M=256, K=512, A=None, B=None, r=0):
+        return f(vp(X), vp(W), None, vp(A), vp(B), M, 512, K, r, 0, vp(Y), vp(ws), ws_bytes, None)
+
+    assert call(X=None) == lynx.LYNX_ERR_INVALID_ARG
+    assert call(Y=None) == lynx.LYNX_ERR_INVALID_ARG
+    assert call(ws=None) == lynx.LYNX_ERR_INVALID_ARG
+    assert call(A=P) == lynx.LYNX_ERR_INVALID_ARG
+    assert call(K=100) == lynx.LYNX_ERR_UNSUPPORTED_SHAPE
+    assert call(M=0) == lynx.LYNX_ERR_UNSUPPORTED_SHAPE
+    assert call(ws=P + 8) == lynx.LYNX_ERR_MISALIGNED
+    assert call(ws_bytes=need - 1) == lynx.LYNX_ERR_WORKSPACE_TOO_SMALL
+
+
 def test_sparse_gemm_argument_errors(lib):
     f = lib.lynx_sparse_gemm
     assert f(vp(P), None, None, vp(P), None, None, 128, 256, 512, 0, vp(P), None) == \
