@@ -73,3 +73,27 @@ def test_graph_layers_match_oracle(sweep_and_plan):
                                      skip=inp["skip"], want_sx=True)
         worst, fro = helpers.y_tolerance_check(y, y_ref, sx, helpers.f32(inp["W"]).astype(np.float64))
         assert worst <= 1.0 and fro <= 5e-3, (plan[i][:2], worst, fro)
+
+
+@pytest.mark.parametrize("layer", [0, 3])  # qkv 3072->9216 and down 12288->3072 (GELU inputs)
+@pytest.mark.parametrize("skip", [False, True])
+def test_full_size_sweep_layer_sampled_rows(layer, skip):
+    """One linear of the sweep at its full size (M = 8192), in the launch
+    configuration the sweep times, on sampled rows; the dense path too."""
+    torch.cuda.set_device(0)
+    lynx.lynx_check_error()
+    _b, _n, M, K, N, kind, _skip, seed = workloads.sweep_plan()[layer]
+    inp = workloads.make_linear_inputs(M, K, N, seed=seed, x_kind=kind)
+    dev = lambda bits: torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to("cuda:0")
+    Y = lynx.lynx_linear(dev(inp["X"]), dev(inp["W"]), dev(inp["bias"]), dev(inp["A"]), dev(inp["B"]),
+                         skip_sparsify=skip)
+    torch.cuda.synchronize()
+    st, code = lynx.lynx_check_error()
+    assert st == lynx.LYNX_OK, (st, code)
+    rng = np.random.default_rng(layer * 2 + int(skip))
+    rows = np.unique(np.concatenate([[0, 255, 256, M - 1], rng.choice(M, 20, replace=False)]))
+    y = helpers.f32(host(Y)).astype(np.float64)[rows]
+    y_ref, _, sx = oracle.linear(inp["X"][rows], inp["W"], inp["bias"], inp["A"], inp["B"], skip=skip,
+                                 want_sx=True)
+    worst, fro = helpers.y_tolerance_check(y, y_ref, sx, helpers.f32(inp["W"]).astype(np.float64))
+    assert worst <= 1.0 and fro <= 5e-3, (layer, skip, worst, fro)
