@@ -82,10 +82,113 @@ struct __align__(1024) PairSmem {
   uint64_t acc_full;           // each CTA's epilogue waits on its own
   uint64_t acc_empty;          // used in the leader CTA (both CTAs' epilogues arrive)
   uint64_t drain;
+  uint64_t fin_done;           // every CTA's rows of s and T are written (fused combining)
   float bias_s[256];
   uint32_t tmem_base;
   volatile uint32_t abort_flag;
 };
+
+// s of row `row` from the sparsify pass's K-range partials, summed in the fixed
+// order j = 0, 1, ...: the same arithmetic as finalize_kernel.
+__device__ __forceinline__ float row_scale_from_partials(const float2* lpart, int64_t M, int split,
+                                                         int64_t row) {
+  float2 v[kMaxSplit];
+#pragma unroll
+  for (int j = 0; j < kMaxSplit; ++j)
+    if (j < split) v[j] = __ldcg(lpart + static_cast<size_t>(j) * M + row);
+  float la = 0.f, lk = 0.f;
+#pragma unroll
+  for (int j = 0; j < kMaxSplit; ++j) {
+    if (j < split) {
+      la = __fadd_rn(la, v[j].x);
+      lk = __fadd_rn(lk, v[j].y);
+    }
+  }
+  return (lk == 0.f) ? 1.f : __fdiv_rn(la, lk);
+}
+
+// This CTA's slice of rows: s, and T written as bf16(T / s) (fin_mode 1) or
+// bf16(T) (fin_mode 2), T summed over the K ranges in the fixed order.  256
+// threads, 8 per row, 8 columns of T each.
+__device__ __forceinline__ void finalize_slice(const GemmLaunch& p, uint32_t et) {
+  const int64_t per = (p.M + gridDim.x - 1) / gridDim.x;
+  const int64_t first = static_cast<int64_t>(blockIdx.x) * per;
+  const int64_t last = (first + per < p.M) ? first + per : p.M;
+  const uint32_t sub = et & 7u;
+  for (int64_t row = first + (et >> 3); row < last; row += 32) {
+    float s = 1.f;
+    if (p.fin_mode == 1) {
+      s = row_scale_from_partials(p.fin_lpart, p.M, p.fin_split, row);
+      if (sub == 0) p.fin_scale[row] = s;
+    }
+    float4 v[kMaxSplit][2];
+#pragma unroll
+    for (int j = 0; j < kMaxSplit; ++j) {
+      if (j < p.fin_split) {
+        const float4* src = reinterpret_cast<const float4*>(
+            p.fin_tpart + (static_cast<size_t>(j) * p.M + row) * kLoraRank + 8 * sub);
+        v[j][0] = __ldcg(src);
+        v[j][1] = __ldcg(src + 1);
+      }
+    }
+    float a[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) a[e] = 0.f;
+#pragma unroll
+    for (int j = 0; j < kMaxSplit; ++j) {
+      if (j < p.fin_split) {
+        a[0] = __fadd_rn(a[0], v[j][0].x);
+        a[1] = __fadd_rn(a[1], v[j][0].y);
+        a[2] = __fadd_rn(a[2], v[j][0].z);
+        a[3] = __fadd_rn(a[3], v[j][0].w);
+        a[4] = __fadd_rn(a[4], v[j][1].x);
+        a[5] = __fadd_rn(a[5], v[j][1].y);
+        a[6] = __fadd_rn(a[6], v[j][1].z);
+        a[7] = __fadd_rn(a[7], v[j][1].w);
+      }
+    }
+    uint32_t pk[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      float x0 = a[2 * e], x1 = a[2 * e + 1];
+      if (p.fin_mode == 1) {
+        x0 = __fdiv_rn(x0, s);
+        x1 = __fdiv_rn(x1, s);
+      }
+      __nv_bfloat162 h = __floats2bfloat162_rn(x0, x1);
+      pk[e] = *reinterpret_cast<uint32_t*>(&h);
+    }
+    *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.fin_t) + row * kLoraRank + 8 * sub) =
+        make_uint4(pk[0], pk[1], pk[2], pk[3]);
+  }
+}
+
+// Each CTA publishes the call's epoch in its own word once its slice is
+// written; the words of an earlier call, of an aborted one, or whatever the
+// workspace held hold other values, so they need no reset.  (A single counter
+// updated by compare-and-swap from every CTA serialised them badly.)
+__device__ __forceinline__ void publish_finalized(const GemmLaunch& p) {
+  asm volatile("st.release.gpu.global.u64 [%0], %1;"
+               ::"l"(p.fin_counter + blockIdx.x), "l"(p.fin_epoch) : "memory");
+}
+
+// The epilogue threads of each CTA wait (bounded) until every CTA of this call
+// has published its slice: thread i watches word i (and i + 256, ...), so the
+// whole grid is checked in one round of loads; a single acquire fence follows.
+__device__ __forceinline__ bool wait_all_finalized(const GemmLaunch& p, uint32_t et) {
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t c = et; c < gridDim.x; c += kEpiThreads) {
+    for (;;) {
+      unsigned long long v;
+      asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p.fin_counter + c) : "memory");
+      if (v == p.fin_epoch) break;
+      if (globaltimer_ns() - t0 > kWaitLimitNs) return false;
+      __nanosleep(64);
+    }
+  }
+  asm volatile("fence.acq_rel.gpu;" ::: "memory");
+  return true;
+}
 
 // tiles walk M first inside a group of `group_m` pair-rows (sized on the host so
 // that the group's A rows stay resident in L2 while W streams once per group)
@@ -130,6 +233,7 @@ lynx_gemm_pair_kernel(const __grid_constant__ GemmLaunch p) {
     mbar_init(&sm.acc_full, 1);
     mbar_init(&sm.acc_empty, 2 * 8);
     mbar_init(&sm.drain, 1);
+    mbar_init(&sm.fin_done, 1);
     sm.abort_flag = 0u;
     fence_mbar_init();
   }
@@ -157,6 +261,7 @@ lynx_gemm_pair_kernel(const __grid_constant__ GemmLaunch p) {
       }
       uint32_t g = 0;
       bool ok = !p.stall_test;
+      bool fin_ready = p.fin_mode == 0;
       for (int tile = cluster_id; ok && tile < ntiles; tile += nclusters) {
         int pm, nb;
         pair_tile_coords(tile, ntm2, ntn, p.group_m, pm, nb);
@@ -194,6 +299,19 @@ lynx_gemm_pair_kernel(const __grid_constant__ GemmLaunch p) {
             }
           } else {
             const int l = kit - nk;
+            if (!fin_ready) {
+              // T of every row is written (by the epilogue warps' round of checks)
+              if (sm.abort_flag || !mbar_wait(&sm.fin_done, 0)) {
+                if (!sm.abort_flag) {
+                  record_error(p.status, kDevTimeoutFinalize);
+                  sm.abort_flag = 1u;
+                }
+                ok = false;
+                break;
+              }
+              asm volatile("fence.proxy.async.global;" ::: "memory");  // T is then read by TMA
+              fin_ready = true;
+            }
             if (leader) mbar_arrive_expect_tx(&sm.full[slot], 2u * (C::kLoraABytes + C::kLoraBBytes));
             tma_load_2d_pair(st, &p.tm_t, lead_full, l * 32, row0);
             tma_load_2d_pair(st + C::kABytes, &p.tm_lb, lead_full, l * 32, col0);
@@ -325,6 +443,23 @@ lynx_gemm_pair_kernel(const __grid_constant__ GemmLaunch p) {
     const uint32_t et = threadIdx.x - 64u;     // 0..255
     const __nv_bfloat16* bias = static_cast<const __nv_bfloat16*>(p.bias);
     const uint32_t lead_acc_empty = mapa_shared(smem_u32(&sm.acc_empty), 0);
+    if (p.fin_mode != 0) {
+      // before the first accumulator is ready: this CTA's rows of s and T
+      finalize_slice(p, et);
+      __threadfence();
+      named_bar_sync(kBarEpilogue, kEpiThreads);
+      if (et == 0) publish_finalized(p);
+      // then every other CTA's slice: the producer loads T once this is done
+      const bool all = wait_all_finalized(p, et);
+      if (named_bar_red_or(kBarEpilogue, kEpiThreads, !all)) {
+        if (et == 0 && !sm.abort_flag) {
+          record_error(p.status, kDevTimeoutFinalize);
+          sm.abort_flag = 1u;
+        }
+      } else if (et == 0) {
+        mbar_arrive(&sm.fin_done);
+      }
+    }
     int acc_count = 0;
     for (int tile = cluster_id; tile < ntiles; tile += nclusters, ++acc_count) {
       int pm, nb;
@@ -337,7 +472,13 @@ lynx_gemm_pair_kernel(const __grid_constant__ GemmLaunch p) {
         const int64_t n = n_base + et;
         sm.bias_s[et] = (bias != nullptr && n < p.N) ? __bfloat162float(bias[n]) : 0.f;
       }
-      const float s = (p.row_scale != nullptr && row_ok) ? p.row_scale[grow] : 1.f;
+      // s of the row: with the fused combining step, written by the slice's
+      // owner before this thread's round of checks (read past L1)
+      float s = 1.f;
+      if (row_ok) {
+        if (p.fin_mode == 1) s = __ldcg(p.fin_scale + grow);
+        else if (p.row_scale != nullptr) s = p.row_scale[grow];
+      }
       bool ok = !sm.abort_flag;
       if (ok && !mbar_wait(&sm.acc_full, static_cast<uint32_t>(acc_count) & 1u)) {
         record_error(p.status, kDevTimeoutAccum);

@@ -6,6 +6,7 @@
 #include <atomic>
 #include <cstring>
 #include <mutex>
+#include <random>
 
 #include "lynx.h"
 #include "lynx_internal.h"
@@ -133,8 +134,12 @@ inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 
 
 inline size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
+// The pair GEMM's grid (at most the SM count) must fit the completion words of
+// its fused partial-combining step in the workspace.
+constexpr int kMaxGemmCtas = 1024;
+
 struct WorkspaceLayout {
-  size_t vals, meta, scale, t, lpart, tpart, total;
+  size_t vals, meta, scale, t, lpart, tpart, counter, total;
 };
 
 // lynx_linear's workspace: kept values | metadata | s | T (or T/s) | partials
@@ -148,7 +153,8 @@ WorkspaceLayout workspace_layout(int64_t M, int64_t K, int64_t r) {
   w.t = align256(w.scale + m * 4);
   w.lpart = align256(w.t + m * kLoraRank * 2);
   w.tpart = align256(w.lpart + static_cast<size_t>(kMaxSplit) * m * 8);
-  w.total = align256(w.tpart + static_cast<size_t>(kMaxSplit) * m * kLoraRank * 4);
+  w.counter = align256(w.tpart + static_cast<size_t>(kMaxSplit) * m * kLoraRank * 4);
+  w.total = align256(w.counter + static_cast<size_t>(kMaxGemmCtas) * 8);  // one word per GEMM CTA
   return w;
 }
 
@@ -186,9 +192,35 @@ lynx_status map_cuda(cudaError_t e) { return e == cudaSuccess ? LYNX_OK : LYNX_E
 
 int gemm_bn(int64_t N) { return N >= 1024 ? 256 : 128; }
 
+// Call tags of the fused partial-combining step: unique within the process
+// (48-bit, from a random start), so a completion word left by an earlier call,
+// an aborted one or unrelated data is never taken for this call's.
+std::atomic<unsigned long long> g_epoch{0};
+std::once_flag g_epoch_once;
+
+unsigned long long next_epoch() {
+  std::call_once(g_epoch_once, []() {
+    std::random_device rd;
+    const unsigned long long seed = (static_cast<unsigned long long>(rd()) << 32) ^ rd();
+    g_epoch.store(seed & ((1ull << 47) - 1));
+  });
+  return g_epoch.fetch_add(1) & ((1ull << 48) - 1);
+}
+
+// The pair GEMM combines the sparsify pass's partials itself (no finalize_kernel).
+struct FusedFinalize {
+  int mode = 0;  // 1: s and bf16(T / s); 2: bf16(T)
+  int split = 1;
+  const float2* lpart = nullptr;
+  const float* tpart = nullptr;
+  float* scale = nullptr;
+  void* t = nullptr;
+  unsigned long long* counter = nullptr;
+};
+
 lynx_status run_sparsify(DeviceState* ds, const void* X, const void* A, int64_t M, int64_t K,
                          void* vals, void* meta, float* row_scale, void* t_out, float2* lpart,
-                         float* tpart, int mode, cudaStream_t stream) {
+                         float* tpart, int mode, cudaStream_t stream, bool skip_finalize = false) {
   SparsifyLaunch p;
   std::memset(&p, 0, sizeof(p));
   if (!encode_bf16_2d(&p.tm_x, X, K, M, K * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B))
@@ -215,6 +247,7 @@ lynx_status run_sparsify(DeviceState* ds, const void* X, const void* A, int64_t 
   p.boxes_per_cta = static_cast<int>(K / 64 / p.split);
   p.kblocks = static_cast<int>((K + 127) / 128);
   p.stall_test = g_stall.load();
+  p.skip_finalize = skip_finalize ? 1 : 0;
   p.status = ds->status;
   return map_cuda(launch_sparsify(p, stream));
 }
@@ -227,7 +260,8 @@ bool use_pair_kernel(int64_t M, int64_t N, int64_t K) {
 
 lynx_status run_gemm(DeviceState* ds, const void* a_src, bool sparse, const void* meta,
                      const float* row_scale, const void* T, const void* W, const void* bias,
-                     const void* B, int64_t M, int64_t N, int64_t K, void* Y, cudaStream_t stream) {
+                     const void* B, int64_t M, int64_t N, int64_t K, void* Y, cudaStream_t stream,
+                     const FusedFinalize* fin = nullptr) {
   GemmLaunch p;
   std::memset(&p, 0, sizeof(p));
   const bool pair = use_pair_kernel(M, N, K);
@@ -281,6 +315,16 @@ lynx_status run_gemm(DeviceState* ds, const void* a_src, bool sparse, const void
     int64_t gm = (40ll << 20) / (a_row_bytes > 0 ? a_row_bytes : 1);
     gm = gm < 1 ? 1 : (gm > ntm2 ? ntm2 : gm);
     p.group_m = static_cast<int>(gm);
+    if (fin != nullptr && fin->mode != 0) {
+      p.fin_mode = fin->mode;
+      p.fin_split = fin->split;
+      p.fin_lpart = fin->lpart;
+      p.fin_tpart = fin->tpart;
+      p.fin_scale = fin->scale;
+      p.fin_t = fin->t;
+      p.fin_counter = fin->counter;
+      p.fin_epoch = next_epoch();
+    }
     return map_cuda(launch_gemm_pair(p, stream));
   }
   const int64_t tiles = ((M + 127) / 128) * ((N + bn - 1) / bn);
@@ -433,25 +477,37 @@ int lynx_linear(const void* X, const void* W, const void* bias, const void* A, c
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   void* t_buf = lora ? ws + wl.t : nullptr;
+  // with the CTA-pair GEMM, the GEMM itself combines the pass's K-range partials
+  const bool fused = use_pair_kernel(M, N, K) && (!skip_sparsify || lora) && ds->sms <= kMaxGemmCtas;
+  FusedFinalize fin;
+  if (fused) {
+    fin.mode = skip_sparsify ? 2 : 1;
+    fin.split = choose_sparsify_split(M, K, ds->sms);
+    fin.lpart = reinterpret_cast<const float2*>(ws + wl.lpart);
+    fin.tpart = reinterpret_cast<const float*>(ws + wl.tpart);
+    fin.scale = reinterpret_cast<float*>(ws + wl.scale);
+    fin.t = t_buf != nullptr ? t_buf : ws + wl.t;
+    fin.counter = reinterpret_cast<unsigned long long*>(ws + wl.counter);
+  }
   if (!skip_sparsify) {
     st = run_sparsify(ds, X, A, M, K, ws + wl.vals, ws + wl.meta,
                       reinterpret_cast<float*>(ws + wl.scale), t_buf,
                       reinterpret_cast<float2*>(ws + wl.lpart), reinterpret_cast<float*>(ws + wl.tpart),
-                      kModeSelect | (lora ? kModeLora : 0), s);
+                      kModeSelect | (lora ? kModeLora : 0), s, fused);
     if (st != LYNX_OK) return st;
     if (void* ev = g_split_event.load())
       if (cudaEventRecord(static_cast<cudaEvent_t>(ev), s) != cudaSuccess) return LYNX_ERR_CUDA;
     return run_gemm(ds, ws + wl.vals, true, ws + wl.meta, reinterpret_cast<const float*>(ws + wl.scale),
-                    t_buf, W, bias, B, M, N, K, Y, s);
+                    t_buf, W, bias, B, M, N, K, Y, s, fused ? &fin : nullptr);
   }
   if (lora) {
     st = run_sparsify(ds, X, A, M, K, nullptr, nullptr, nullptr, t_buf, nullptr,
-                      reinterpret_cast<float*>(ws + wl.tpart), kModeLora, s);
+                      reinterpret_cast<float*>(ws + wl.tpart), kModeLora, s, fused);
     if (st != LYNX_OK) return st;
   }
   if (void* ev = g_split_event.load())
     if (cudaEventRecord(static_cast<cudaEvent_t>(ev), s) != cudaSuccess) return LYNX_ERR_CUDA;
-  return run_gemm(ds, X, false, nullptr, nullptr, t_buf, W, bias, B, M, N, K, Y, s);
+  return run_gemm(ds, X, false, nullptr, nullptr, t_buf, W, bias, B, M, N, K, Y, s, fused ? &fin : nullptr);
 }
 
 size_t lynx_linear_host_workspace_bytes(int64_t M, int64_t N, int64_t K, int64_t r) {

@@ -39,6 +39,7 @@ struct SparsifyLaunch {
   int boxes_per_cta;    // 64-column boxes each CTA covers
   int kblocks;          // metadata blocks per row block: ceil(K/128)
   int stall_test;       // test-only: the producer never loads, waits must time out
+  int skip_finalize;    // the GEMM that follows combines the partials (finalize_kernel not launched)
   uint32_t* status;     // device status word (first error code wins)
 };
 
@@ -87,6 +88,21 @@ struct GemmLaunch {
   int group_m;          // tile rows (of 128 or of 256 for CTA pairs) per raster group
   int stall_test;
   uint32_t* status;
+  // Combining the sparsify pass's K-range partials inside the pair GEMM (instead
+  // of finalize_kernel): fin_mode 1 = s and bf16(T / s), 2 = bf16(T) only, 0 =
+  // off.  Each CTA's epilogue warps combine a slice of the rows before their
+  // first tile and then write fin_epoch into fin_counter[blockIdx.x] (the epoch
+  // is unique per call, so the words need no initial value).  Then they wait for
+  // every CTA's word and signal their producer, which loads T only after that;
+  // the epilogue then reads each row's s from fin_scale.
+  int fin_mode;
+  int fin_split;
+  const float2* fin_lpart;
+  const float* fin_tpart;
+  float* fin_scale;
+  void* fin_t;
+  unsigned long long* fin_counter;  // one word per CTA of the grid
+  unsigned long long fin_epoch;
 };
 
 cudaError_t launch_gemm(const GemmLaunch& p, cudaStream_t stream);       // 128 x BN tiles, 1 CTA

@@ -19,6 +19,7 @@ enum DeviceError : uint32_t {
   kDevTimeoutEmpty = 0x102,    // producer gave up waiting for a free stage
   kDevTimeoutAccum = 0x103,    // MMA / epilogue gave up waiting on the accumulator
   kDevTimeoutDrain = 0x104,    // gave up waiting for copies in flight at exit
+  kDevTimeoutFinalize = 0x105, // gave up waiting for the row partials to be combined
   kDevTimeoutTest = 0x1FF,     // the test-only stall switch fired
 };
 

@@ -473,7 +473,7 @@ cudaError_t launch_sparsify(const SparsifyLaunch& p, cudaStream_t stream) {
   // pattern of all-zero rows, so a CTA pair of the GEMM never reads garbage
   const dim3 grid(static_cast<unsigned>(p.split), static_cast<unsigned>(meta_row_blocks(p.M)), 1);
   cudaError_t e = launch_after_previous(sparsify_kernel, grid, dim3(kThreads), smem, stream, p);
-  if (e != cudaSuccess) return e;
+  if (e != cudaSuccess || p.skip_finalize) return e;
   const bool do_sel = (p.mode & kModeSelect) != 0;
   const bool do_lora = (p.mode & kModeLora) != 0;
   const bool scaled = (p.mode & kModeScaled) != 0;
