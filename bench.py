@@ -38,15 +38,25 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # DRAM bytes (read + write) per launch of the sparse GEMM kernel, from one ncu
 # capture of the kernel as it stands (dram__bytes_read.sum + dram__bytes_write.sum);
 # a workload that has not been captured reports null.
-GEMM_DRAM_TRAFFIC = {"mlp_up": 93.91e6 + 82.72e6}
+GEMM_DRAM_TRAFFIC = {"mlp_up": 102.96e6 + 84.07e6}
 
-# kernels one sparse lynx_linear call launches: sparsify pass, per-row finalize, GEMM
-LAUNCHES_PER_LINEAR = 3
+def uses_pair_gemm(M, N, K):
+    """The library's choice: the CTA-pair GEMM unless the shape cannot feed it."""
+    return M > 128 and N >= 256 and K % 128 == 0
+
+
+def launches_per_linear(M, N, K, skip=False, lora=True):
+    """Kernels one lynx_linear call launches: the sparsify pass (or, on the dense
+    path, the LoRA-down pass), a finalize kernel unless the pair GEMM combines
+    the pass's partials itself, and the GEMM."""
+    if skip and not lora:
+        return 1
+    return 2 if uses_pair_gemm(M, N, K) else 3
 
 
 def gemm_kernel_name(M, N, K):
     """Name of the GEMM kernel the library picks for a sparse call of this shape."""
-    if M > 128 and N >= 256 and K % 128 == 0:
+    if uses_pair_gemm(M, N, K):
         return "lynx_gemm_pair_kernel<1> (CTA pair, 256x256 tiles)"
     return f"lynx_gemm_kernel<{256 if N >= 1024 else 128},1>"
 
@@ -439,7 +449,7 @@ def run_lynx(args):
                 "ms_per_step": e2e_ms,
                 "note": "lynx_linear_host on pinned host X and Y: the copies in, the layer and the "
                         "copies out inside each step, overlapped over row chunks; weights resident"},
-        "gpu_launches": LAUNCHES_PER_LINEAR * args.steps,
+        "gpu_launches": launches_per_linear(M, N, K) * args.steps,
         "clocks": clock_info,
     }
 
@@ -453,6 +463,11 @@ def run_lynx(args):
     if rank == 0:
         print(json.dumps(result), flush=True)
     return 0
+
+
+def _mkn(t):
+    M, K, N = t["shape"]
+    return M, N, K
 
 
 def run_sweep(args):
@@ -565,8 +580,8 @@ def run_sweep(args):
         "speedup_vs_dense_bf16": dense_ms / ms_step,
         "breakdown_ms": {"sweep_graph": ms_step, "sweep_eager": eager_ms,
                          "dense_torch_matmul_graph": dense_ms},
-        # per layer: sparsify pass, finalize, GEMM (a dense layer without LoRA: the GEMM)
-        "gpu_launches": args.steps * sum(1 if t["skip"] and t["A"] is None else 3
+        "gpu_launches": args.steps * sum(launches_per_linear(*_mkn(t), skip=t["skip"],
+                                                             lora=t["A"] is not None)
                                          for t in sweep.layers),
         "clocks": clock_info,
     }
