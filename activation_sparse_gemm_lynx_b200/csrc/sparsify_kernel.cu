@@ -151,11 +151,13 @@ sparsify_kernel(const __grid_constant__ SparsifyLaunch p) {
     sm.abort_flag = 0u;
     fence_mbar_init();
   }
-  // The first stages' loads leave before the rest of the prologue (TMEM
-  // allocation, the block barrier): the first box is the one whose latency
-  // nothing else hides.  They wait for the previous kernel like every access
-  // to X below.
-  const int preissued = (nboxes < kStages) ? nboxes : kStages;
+  // The first box's loads leave before the rest of the prologue (TMEM
+  // allocation, the block barrier): its latency is the one nothing else hides.
+  // The other stages' loads follow only once it has landed, so that the first
+  // wave of requests from the whole grid is one box per CTA and each CTA can
+  // start computing while the rest streams in.  The loads wait for the previous
+  // kernel like every access to X below.
+  const int preissued = (nboxes < 1) ? nboxes : 1;
   if (threadIdx.x == 0 && !p.stall_test) {
     tma_prefetch_desc(&p.tm_x);
     if (do_lora) tma_prefetch_desc(&p.tm_a);
@@ -217,6 +219,10 @@ sparsify_kernel(const __grid_constant__ SparsifyLaunch p) {
             set_abort(sm, p.status, kDevTimeoutEmpty);
             break;
           }
+        }
+        if (b == preissued && b < kStages && preissued > 0 && !mbar_wait(&sm.full[0], 0)) {
+          set_abort(sm, p.status, kDevTimeoutFull);
+          break;
         }
         if (b >= preissued && b < nboxes) {
           mbar_arrive_expect_tx(&sm.full[slot], tx);
