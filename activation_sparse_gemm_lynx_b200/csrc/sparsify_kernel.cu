@@ -188,8 +188,9 @@ sparsify_kernel(const __grid_constant__ SparsifyLaunch p) {
     // ------------------------------------------------------------ producer
     // Loads box b into stage b % kStages once box b - kStages has left it.
     // The row threads' release of a stage also means that the kept values of
-    // that box are staged, so the same thread then issues their TMA store and,
-    // once the store has read its buffer, hands the buffer back (vfree).
+    // that box are staged, so the same thread then issues their TMA store and
+    // hands back the buffer of the previous box's store, which has read it by
+    // then (vfree).  The last box's buffer is not needed again.
     if (lane == 0) {
       if (do_sel) tma_prefetch_desc(&p.tm_vals);
       const uint32_t tx = kXTileBytes + (do_lora ? kATileBytes : 0u);
@@ -211,9 +212,13 @@ sparsify_kernel(const __grid_constant__ SparsifyLaunch p) {
               tma_store_2d(&p.tm_vals, sm.vstage[prev & 1], static_cast<int32_t>((kcol0 + 64 * prev) / 2),
                            static_cast<int32_t>(mb * 128));
               bulk_commit();
-              bulk_wait_read_all();
+              // the store of box prev - 1 has read its buffer (this one may still
+              // be reading): hand that buffer back, without waiting on this store
+              bulk_wait_read_le1();
+              if (prev > 0) mbar_arrive(&sm.vfree[(prev - 1) & 1]);
+            } else {
+              mbar_arrive(&sm.vfree[prev & 1]);
             }
-            mbar_arrive(&sm.vfree[prev & 1]);
           }
           if (do_lora && !mbar_wait(&sm.mma_done[slot], pph)) {
             set_abort(sm, p.status, kDevTimeoutEmpty);
