@@ -24,6 +24,7 @@ import datetime
 import json
 import math
 import os
+import platform
 import statistics
 import sys
 import threading
@@ -219,13 +220,43 @@ def calibrate_oracle_rows(inp, target_s, M):
     return rows, cores
 
 
+def cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return platform.processor() or "unknown"
+
+
+def single_thread_sample(inp, shape, target_s):
+    """The same oracle on one thread, on whole rows for about `target_s`."""
+    import oracle
+
+    cores = oracle.num_threads()
+    oracle.set_num_threads(1)
+    try:
+        rows = 1
+        t = oracle_sample(inp, rows)
+        rows = min(shape.M, max(1, int(rows * target_s / max(t, 1e-3))))
+        t = oracle_sample(inp, rows)
+    finally:
+        oracle.set_num_threads(cores)
+    return {"value": 2.0 * rows * shape.N * shape.K / t / 1e12, "unit": "TFLOP/s", "cores": 1,
+            "sample": f"{rows} token rows, {t:.1f} s"}
+
+
 def cpu_baseline(inp, shape, target_s):
     rows, cores = calibrate_oracle_rows(inp, target_s, shape.M)
     t = oracle_sample(inp, rows)
     flops = 2.0 * rows * shape.N * shape.K
     return {"value": flops / t / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
             "sample": f"{rows} of {shape.M} token rows of {shape.name} (rows are independent), "
-                      f"full N={shape.N} and K={shape.K}, fp64 C oracle, {t:.1f} s"}
+                      f"full N={shape.N} and K={shape.K}, fp64 C oracle, {t:.1f} s",
+            "cpu": cpu_model(),
+            "single_thread": single_thread_sample(inp, shape, min(3.0, target_s / 4))}
 
 
 # ---------------------------------------------------------------------------
@@ -265,7 +296,7 @@ def run_reference(args):
         "config": {"workload": workload_desc(shape), "M": shape.M, "N": shape.N, "K": shape.K,
                    "r": shape.r, "rows_per_step": rows},
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
-                         "sample": sample},
+                         "sample": sample, "cpu": cpu_model()},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
         "gpu_launches": 0,
     }

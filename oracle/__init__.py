@@ -39,8 +39,9 @@ def _load():
         lib.oracle_select_groups.argtypes = [p, i64, p, p]
         lib.oracle_sparsify.argtypes = [p, i64, i64, p, p, p, p]
         lib.oracle_linear.argtypes = [p, p, p, p, p, i64, i64, i64, i64, ctypes.c_int, p, p, p]
+        lib.oracle_set_threads.argtypes = [ctypes.c_int]
         for f in (lib.oracle_bf16_rne, lib.oracle_select_groups, lib.oracle_sparsify,
-                  lib.oracle_linear):
+                  lib.oracle_linear, lib.oracle_set_threads):
             f.restype = None
         _lib = lib
     return _lib
@@ -134,7 +135,21 @@ def linear(X, W, bias=None, A=None, B=None, skip=False, want_sx=False):
     return Y, T, SX
 
 
+_threads = None
+
+
 def num_threads():
-    """Threads the oracle's OpenMP loops use (OMP_NUM_THREADS or all cores)."""
+    """Threads the oracle's OpenMP loops use (set_num_threads, else
+    OMP_NUM_THREADS, else all cores)."""
+    if _threads is not None:
+        return _threads
     env = os.environ.get("OMP_NUM_THREADS")
     return int(env) if env else os.cpu_count()
+
+
+def set_num_threads(n):
+    """Run the oracle's parallel loops on `n` threads from now on (timing only:
+    each output element is computed by one thread, in a fixed order)."""
+    global _threads
+    _load().oracle_set_threads(int(n))
+    _threads = int(n)

@@ -47,6 +47,9 @@
 #include <stdint.h>
 #include <stdlib.h>
 #include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
 
 typedef uint16_t bf16_bits;
 
@@ -233,4 +236,15 @@ void oracle_linear(const bf16_bits *X, const bf16_bits *W, const bf16_bits *bias
     free(vrow);
     free(mrow);
   }
+}
+
+/* Threads used by the parallel loops above from now on (timing only; the
+ * results do not depend on it: every output element is computed by one thread
+ * in a fixed order). */
+void oracle_set_threads(int n) {
+#ifdef _OPENMP
+  if (n > 0) omp_set_num_threads(n);
+#else
+  (void)n;
+#endif
 }
