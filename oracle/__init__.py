@@ -17,6 +17,8 @@ Place for Diffusion Models" (qingkeai.online article, sections 02-03):
 * :func:`linear` -- Y = S(X) W^T + bias + (X A^T) B^T in fp64 (S(X) := X for
   a skipped layer).
 * :func:`bf16_rne` -- IEEE round-to-nearest-even fp32 -> bf16.
+* :func:`gelu_tanh` -- GELU (tanh form) in fp64, the activation the library can
+  apply to a layer's output (not part of the pages' method).
 """
 import ctypes
 import os
@@ -40,8 +42,9 @@ def _load():
         lib.oracle_sparsify.argtypes = [p, i64, i64, p, p, p, p]
         lib.oracle_linear.argtypes = [p, p, p, p, p, i64, i64, i64, i64, ctypes.c_int, p, p, p]
         lib.oracle_set_threads.argtypes = [ctypes.c_int]
+        lib.oracle_gelu_tanh.argtypes = [p, i64, p]
         for f in (lib.oracle_bf16_rne, lib.oracle_select_groups, lib.oracle_sparsify,
-                  lib.oracle_linear, lib.oracle_set_threads):
+                  lib.oracle_linear, lib.oracle_set_threads, lib.oracle_gelu_tanh):
             f.restype = None
         _lib = lib
     return _lib
@@ -133,6 +136,16 @@ def linear(X, W, bias=None, A=None, B=None, skip=False, want_sx=False):
     _load().oracle_linear(_ptr(X), _ptr(W), _ptr(bias), _ptr(A), _ptr(B), M, N, K, r,
                           1 if skip else 0, _ptr(Y), _ptr(T), _ptr(SX))
     return Y, T, SX
+
+
+def gelu_tanh(v):
+    """GELU, tanh form (Hendrycks & Gimpel), elementwise in fp64:
+    v/2 (1 + tanh(sqrt(2/pi) (v + 0.044715 v^3))).  The activation the library
+    can apply to a layer's output; compose as gelu_tanh(linear(...)[0])."""
+    a = np.ascontiguousarray(v, dtype=np.float64)
+    out = np.empty_like(a)
+    _load().oracle_gelu_tanh(_ptr(a), a.size, _ptr(out))
+    return out
 
 
 _threads = None

@@ -30,6 +30,12 @@
  *   - qingkeai section 03.3 (selective layer skipping): skipped layers stay
  *     dense, S(X) := X.
  *
+ *   - An activation on the layer's output (not part of the pages' method; the
+ *     DiT MLP applies it between its up- and down-projections, and the
+ *     library can apply it in the GEMM epilogue): GELU, tanh form
+ *     (Hendrycks & Gimpel, "Gaussian Error Linear Units"),
+ *     gelu(v) = v/2 (1 + tanh(sqrt(2/pi) (v + 0.044715 v^3))), in fp64.
+ *
  * Precision: selection compares magnitudes exactly; the two row sums are fp32
  * sums in increasing k order; s is one IEEE fp32 division; each kept value is
  * one fp32 multiply rounded to nearest even, then rounded to nearest even to
@@ -235,6 +241,18 @@ void oracle_linear(const bf16_bits *X, const bf16_bits *W, const bf16_bits *bias
     free(trow);
     free(vrow);
     free(mrow);
+  }
+}
+
+/* GELU, tanh form, in fp64, for n values.  Written with the identity
+ * (1 + tanh u)/2 = 1/(1 + exp(-2u)), the same function without the
+ * cancellation in 1 + tanh u when u is very negative. */
+void oracle_gelu_tanh(const double *v, int64_t n, double *out) {
+  const double c = sqrt(2.0 / 3.14159265358979323846);
+  for (int64_t i = 0; i < n; ++i) {
+    const double x = v[i];
+    const double u = c * (x + 0.044715 * x * x * x);
+    out[i] = x / (1.0 + exp(-2.0 * u));
   }
 }
 

@@ -313,3 +313,41 @@ def test_worked_examples(oracle_mod, case):
     want = np.array(case["vals"], dtype=np.float32)
     got = f32(r["vals"][0, : K // 2])
     assert np.array_equal(got.view(np.uint32), want.view(np.uint32))  # -0 vs +0 too
+
+
+# --------------------------------------------------------------------------
+# GELU (tanh form), the optional output activation: pinned to torch's own
+# fp64 GELU, to the function's odd-part identity, to its value and slope at 0
+# and to its distance from the exact (erf) GELU it approximates.
+
+def test_gelu_matches_torch_fp64(oracle_mod):
+    v = np.concatenate([np.linspace(-4.0, 8.0, 2401),
+                        np.random.default_rng(7).normal(-0.5, 1.0, 4000).clip(-4.0, None)])
+    want = torch.nn.functional.gelu(torch.from_numpy(v), approximate="tanh").numpy()
+    got = oracle_mod.gelu_tanh(v)
+    # torch evaluates v/2 (1 + tanh u): its own rounding error relative to the
+    # result grows like 1e-16 / (1 + tanh u) = 1e-16 / (2 e^(2u)), about 3e-12
+    # at v = -4 (and 1e-9 at v = -5, where the comparison would test torch)
+    np.testing.assert_allclose(got, want, rtol=1e-11, atol=1e-300)
+
+
+def test_gelu_odd_part_is_identity(oracle_mod):
+    # (1 + tanh u)/2 - (1 - tanh u)/2 = tanh u ... so gelu(v) - gelu(-v) = v
+    v = np.random.default_rng(8).normal(0.0, 3.0, 5000)
+    d = oracle_mod.gelu_tanh(v) - oracle_mod.gelu_tanh(-v)
+    np.testing.assert_allclose(d, v, rtol=1e-13, atol=1e-15)
+
+
+def test_gelu_at_zero_and_tails(oracle_mod):
+    g = oracle_mod.gelu_tanh(np.array([0.0, -1e-6, 1e-6, 40.0, -40.0]))
+    assert g[0] == 0.0
+    # slope 1/2 at the origin
+    assert abs((g[2] - g[1]) / 2e-6 - 0.5) < 1e-9
+    assert g[3] == 40.0 and g[4] == 0.0
+
+
+def test_gelu_tanh_form_is_close_to_erf_gelu(oracle_mod):
+    # the tanh form approximates v * Phi(v); the two stay within 1e-3 everywhere
+    v = np.linspace(-8.0, 8.0, 16001)
+    exact = torch.nn.functional.gelu(torch.from_numpy(v)).numpy()
+    assert np.max(np.abs(oracle_mod.gelu_tanh(v) - exact)) < 1e-3
