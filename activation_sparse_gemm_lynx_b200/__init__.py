@@ -13,12 +13,16 @@ The public entry points mirror the C ABI of ``include/lynx.h``; see
 synthetic inputs used by the tests and the benchmark.
 """
 from .lynx import (  # noqa: F401
+    LYNX_ACT_GELU_TANH,
+    LYNX_ACT_NONE,
     LynxError,
     lynx_check_error,
     lynx_debug_set_stall,
     lynx_linear,
+    lynx_linear_act,
     lynx_linear_dense,
     lynx_linear_host,
+    lynx_linear_host_act,
     lynx_linear_host_workspace_bytes,
     lynx_lora_rank,
     lynx_meta_bytes,

@@ -5,7 +5,8 @@
 // path of layers left dense by selective layer skipping).  T = X A^T is the
 // LoRA down-projection produced by the sparsify pass; the LoRA up-projection
 // runs as two extra dense K=32 steps into the same TMEM accumulator tile, and
-// the bias is added in fp32 before the single bf16 rounding of Y.
+// the bias is added in fp32 before the single bf16 rounding of Y (after an
+// optional activation, GELU tanh form, also in fp32).
 // (RT-Lynx pages: qingkeai.online article section 02, Y = S(X) W^T; section
 // 03.2, LoRA residual; section 03.3, skipped layers; section 04, sparse GEMM
 // and LoRA residual fused into the CUDA kernel.)
@@ -24,6 +25,7 @@
 // Accumulators: 1 TMEM buffer for BN = 256, 2 (double buffered) for BN = 128.
 #include <cuda_bf16.h>
 
+#include "lynx_act.cuh"
 #include "lynx_internal.h"
 #include "lynx_ptx.cuh"
 
@@ -258,7 +260,7 @@ lynx_gemm_kernel(const __grid_constant__ GemmLaunch p) {
     __syncwarp();
   } else {
     // ------------------------------------------------------------ epilogue
-    // Y = bf16(s_row * acc + bias).  Two warps per TMEM lane quarter, each
+    // Y = bf16(act(s_row * acc + bias)).  Two warps per TMEM lane quarter, each
     // draining half of the columns into registers; the TMEM buffer is released
     // before the global stores, so the next tile's MMAs overlap them.
     constexpr int kHalf = BN / 2;
@@ -301,8 +303,12 @@ lynx_gemm_kernel(const __grid_constant__ GemmLaunch p) {
         tmem_ld_wait();
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-          const float a = __fmaf_rn(s, __uint_as_float(r[2 * i]), sm.bias_s[col + 2 * i]);
-          const float b = __fmaf_rn(s, __uint_as_float(r[2 * i + 1]), sm.bias_s[col + 2 * i + 1]);
+          float a = __fmaf_rn(s, __uint_as_float(r[2 * i]), sm.bias_s[col + 2 * i]);
+          float b = __fmaf_rn(s, __uint_as_float(r[2 * i + 1]), sm.bias_s[col + 2 * i + 1]);
+          if (p.act == kActGeluTanh) {
+            a = gelu_tanh(a);
+            b = gelu_tanh(b);
+          }
           __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
           out[16 * c + i] = *reinterpret_cast<uint32_t*>(&h);
         }

@@ -1,5 +1,5 @@
 // gemm_pair_kernel.cu -- the Lynx GEMM on CTA pairs (tcgen05 cta_group::2):
-//   Y[M,N] = bf16( s_row * (S(X) W^T + T' B^T) + bias )
+//   Y[M,N] = bf16( act( s_row * (S(X) W^T + T' B^T) + bias ) )   (act: none or GELU)
 // Same arithmetic as gemm_kernel.cu (see there and the RT-Lynx references),
 // computed on 256 x 256 output tiles by a pair of CTAs on the two SMs of a
 // TPC: each CTA holds 128 rows of A (compressed activations, or X on the dense
@@ -20,7 +20,7 @@
 //               single MMA issuer: tcgen05.cp of both CTAs' metadata, the MMAs,
 //               and commits multicast to both CTAs' "empty" / "acc_full"
 //               barriers.
-//   warps 2-9   epilogue on the CTA's own 128 accumulator rows: s * acc + bias
+//   warps 2-9   epilogue on the CTA's own 128 accumulator rows: act(s * acc + bias)
 //               -> bf16 -> global; releases the accumulator by arriving on the
 //               leader's "acc_empty" barrier.
 //   warp 10     in the leader CTA: waits for each filled stage ("full") and
@@ -31,6 +31,7 @@
 //               not.
 #include <cuda_bf16.h>
 
+#include "lynx_act.cuh"
 #include "lynx_internal.h"
 #include "lynx_ptx.cuh"
 
@@ -203,7 +204,7 @@ __device__ __forceinline__ void pair_tile_coords(int tile, int ntm2, int ntn, in
   nb = in_group / gm;
 }
 
-template <bool SPARSE>
+template <bool SPARSE, int ACT>
 __global__ void __launch_bounds__(kThreads, 1)
 lynx_gemm_pair_kernel(const __grid_constant__ GemmLaunch p) {
   using C = PairCfg<SPARSE>;
@@ -489,8 +490,8 @@ lynx_gemm_pair_kernel(const __grid_constant__ GemmLaunch p) {
       tc_fence_after();
       // The warp's 32 rows x 128 columns of the accumulator go to registers
       // first and the accumulator is handed back at once, so the next tile's
-      // MMAs start while this tile is converted and stored: s * acc + bias ->
-      // bf16 -> 16-column pieces staged in shared memory -> asynchronous bulk
+      // MMAs start while this tile is converted and stored: act(s * acc + bias)
+      // -> bf16 -> 16-column pieces staged in shared memory -> asynchronous bulk
       // tensor stores (rows past M / columns past N are clipped by the TMA)
       const int32_t store_row = static_cast<int32_t>(pm * 256 + rank * 128 + 32 * q);
       uint8_t* my_stage = sm.ystage[warp - 2][0];
@@ -512,8 +513,9 @@ lynx_gemm_pair_kernel(const __grid_constant__ GemmLaunch p) {
 #pragma unroll
           for (int i = 0; i < 8; ++i) {
             const int e = 16 * h + 2 * i;
-            const float a = __fmaf_rn(s, __uint_as_float(r[c][e]), sm.bias_s[col + e]);
-            const float b = __fmaf_rn(s, __uint_as_float(r[c][e + 1]), sm.bias_s[col + e + 1]);
+            const float a = apply_act<ACT>(__fmaf_rn(s, __uint_as_float(r[c][e]), sm.bias_s[col + e]));
+            const float b =
+                apply_act<ACT>(__fmaf_rn(s, __uint_as_float(r[c][e + 1]), sm.bias_s[col + e + 1]));
             __nv_bfloat162 hv = __floats2bfloat162_rn(a, b);
             pk[i] = *reinterpret_cast<uint32_t*>(&hv);
           }
@@ -541,14 +543,14 @@ lynx_gemm_pair_kernel(const __grid_constant__ GemmLaunch p) {
   if (warp == 1) tmem_dealloc_pair(sm.tmem_base, kTmemCols);
 }
 
-template <bool SPARSE>
+template <bool SPARSE, int ACT>
 cudaError_t launch_pair_variant(const GemmLaunch& p, cudaStream_t stream) {
   const size_t smem = sizeof(PairSmem<SPARSE>) + 1024;
   static int configured_device = -1;
   int dev = 0;
   cudaGetDevice(&dev);
   if (configured_device != dev) {
-    cudaError_t e = cudaFuncSetAttribute(lynx_gemm_pair_kernel<SPARSE>,
+    cudaError_t e = cudaFuncSetAttribute(lynx_gemm_pair_kernel<SPARSE, ACT>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
     if (e != cudaSuccess) return e;
@@ -568,13 +570,17 @@ cudaError_t launch_pair_variant(const GemmLaunch& p, cudaStream_t stream) {
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  return cudaLaunchKernelEx(&cfg, lynx_gemm_pair_kernel<SPARSE>, p);
+  return cudaLaunchKernelEx(&cfg, lynx_gemm_pair_kernel<SPARSE, ACT>, p);
 }
 
 }  // namespace
 
 cudaError_t launch_gemm_pair(const GemmLaunch& p, cudaStream_t stream) {
-  return p.sparse ? launch_pair_variant<true>(p, stream) : launch_pair_variant<false>(p, stream);
+  if (p.act == kActGeluTanh)
+    return p.sparse ? launch_pair_variant<true, kActGeluTanh>(p, stream)
+                    : launch_pair_variant<false, kActGeluTanh>(p, stream);
+  return p.sparse ? launch_pair_variant<true, kActNone>(p, stream)
+                  : launch_pair_variant<false, kActNone>(p, stream);
 }
 
 }  // namespace lynx

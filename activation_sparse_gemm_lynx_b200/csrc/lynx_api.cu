@@ -261,7 +261,7 @@ bool use_pair_kernel(int64_t M, int64_t N, int64_t K) {
 lynx_status run_gemm(DeviceState* ds, const void* a_src, bool sparse, const void* meta,
                      const float* row_scale, const void* T, const void* W, const void* bias,
                      const void* B, int64_t M, int64_t N, int64_t K, void* Y, cudaStream_t stream,
-                     const FusedFinalize* fin = nullptr) {
+                     const FusedFinalize* fin = nullptr, int act = kActNone) {
   GemmLaunch p;
   std::memset(&p, 0, sizeof(p));
   const bool pair = use_pair_kernel(M, N, K);
@@ -303,6 +303,7 @@ lynx_status run_gemm(DeviceState* ds, const void* a_src, bool sparse, const void
   p.lora = lora ? 1 : 0;
   p.bn = bn;
   p.stall_test = g_stall.load();
+  p.act = act;
   p.status = ds->status;
   if (pair) {
     const int64_t ntm2 = (M + 255) / 256;
@@ -459,7 +460,15 @@ int lynx_sparsify_noalloc(const void* X, int64_t M, int64_t K, void* vals, void*
 int lynx_linear(const void* X, const void* W, const void* bias, const void* A, const void* B,
                 int64_t M, int64_t N, int64_t K, int64_t r, int skip_sparsify, void* Y,
                 void* workspace, size_t workspace_bytes, void* stream) {
+  return lynx_linear_act(X, W, bias, A, B, M, N, K, r, skip_sparsify, LYNX_ACT_NONE, Y, workspace,
+                         workspace_bytes, stream);
+}
+
+int lynx_linear_act(const void* X, const void* W, const void* bias, const void* A, const void* B,
+                    int64_t M, int64_t N, int64_t K, int64_t r, int skip_sparsify, int act, void* Y,
+                    void* workspace, size_t workspace_bytes, void* stream) {
   if (X == nullptr || W == nullptr || Y == nullptr) return LYNX_ERR_INVALID_ARG;
+  if (act != LYNX_ACT_NONE && act != LYNX_ACT_GELU_TANH) return LYNX_ERR_INVALID_ARG;
   lynx_status st = check_lora(A, B, r);
   if (st != LYNX_OK) return st;
   st = check_shape(M, N, K);
@@ -498,7 +507,7 @@ int lynx_linear(const void* X, const void* W, const void* bias, const void* A, c
     if (void* ev = g_split_event.load())
       if (cudaEventRecord(static_cast<cudaEvent_t>(ev), s) != cudaSuccess) return LYNX_ERR_CUDA;
     return run_gemm(ds, ws + wl.vals, true, ws + wl.meta, reinterpret_cast<const float*>(ws + wl.scale),
-                    t_buf, W, bias, B, M, N, K, Y, s, fused ? &fin : nullptr);
+                    t_buf, W, bias, B, M, N, K, Y, s, fused ? &fin : nullptr, act);
   }
   if (lora) {
     st = run_sparsify(ds, X, A, M, K, nullptr, nullptr, nullptr, t_buf, nullptr,
@@ -507,7 +516,8 @@ int lynx_linear(const void* X, const void* W, const void* bias, const void* A, c
   }
   if (void* ev = g_split_event.load())
     if (cudaEventRecord(static_cast<cudaEvent_t>(ev), s) != cudaSuccess) return LYNX_ERR_CUDA;
-  return run_gemm(ds, X, false, nullptr, nullptr, t_buf, W, bias, B, M, N, K, Y, s, fused ? &fin : nullptr);
+  return run_gemm(ds, X, false, nullptr, nullptr, t_buf, W, bias, B, M, N, K, Y, s, fused ? &fin : nullptr,
+                  act);
 }
 
 size_t lynx_linear_host_workspace_bytes(int64_t M, int64_t N, int64_t K, int64_t r) {
@@ -520,8 +530,16 @@ size_t lynx_linear_host_workspace_bytes(int64_t M, int64_t N, int64_t K, int64_t
 int lynx_linear_host(const void* X_host, const void* W, const void* bias, const void* A, const void* B,
                      int64_t M, int64_t N, int64_t K, int64_t r, int skip_sparsify, void* Y_host,
                      void* workspace, size_t workspace_bytes, void* stream) {
+  return lynx_linear_host_act(X_host, W, bias, A, B, M, N, K, r, skip_sparsify, LYNX_ACT_NONE, Y_host,
+                              workspace, workspace_bytes, stream);
+}
+
+int lynx_linear_host_act(const void* X_host, const void* W, const void* bias, const void* A,
+                         const void* B, int64_t M, int64_t N, int64_t K, int64_t r, int skip_sparsify,
+                         int act, void* Y_host, void* workspace, size_t workspace_bytes, void* stream) {
   if (X_host == nullptr || W == nullptr || Y_host == nullptr || workspace == nullptr)
     return LYNX_ERR_INVALID_ARG;
+  if (act != LYNX_ACT_NONE && act != LYNX_ACT_GELU_TANH) return LYNX_ERR_INVALID_ARG;
   lynx_status st = check_lora(A, B, r);
   if (st != LYNX_OK) return st;
   st = check_shape(M, N, K);
@@ -553,8 +571,8 @@ int lynx_linear_host(const void* X_host, const void* W, const void* bias, const 
         cudaEventRecord(hp->in_done[chunk], hp->in) != cudaSuccess ||
         cudaStreamWaitEvent(s, hp->in_done[chunk], 0) != cudaSuccess)
       return LYNX_ERR_CUDA;
-    st = static_cast<lynx_status>(lynx_linear(x_dev + off_x, W, bias, A, B, mc, N, K, r, skip_sparsify,
-                                              y_dev + off_y, layer_ws, layer_bytes, s));
+    st = static_cast<lynx_status>(lynx_linear_act(x_dev + off_x, W, bias, A, B, mc, N, K, r, skip_sparsify,
+                                                  act, y_dev + off_y, layer_ws, layer_bytes, s));
     if (st != LYNX_OK) return st;
     if (cudaEventRecord(hp->comp_done[chunk], s) != cudaSuccess ||
         cudaStreamWaitEvent(hp->out, hp->comp_done[chunk], 0) != cudaSuccess ||

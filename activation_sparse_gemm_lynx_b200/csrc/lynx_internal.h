@@ -21,6 +21,10 @@ constexpr int kMetaBlockBytes = 2048;  // 128 TMEM lanes x 16 bytes
 // leave as kept and s is applied by the GEMM (T is then written as T / s).
 enum SparsifyMode : int { kModeSelect = 1, kModeLora = 2, kModeScaled = 4 };
 
+// Activation the GEMM epilogue applies to each finished output value (the
+// LYNX_ACT_* values of the public header).
+enum EpilogueAct : int { kActNone = 0, kActGeluTanh = 1 };
+
 constexpr int kMaxSplit = 8;  // K ranges per row block in the sparsify pass
 
 struct SparsifyLaunch {
@@ -87,6 +91,7 @@ struct GemmLaunch {
   int grid;             // persistent CTAs
   int group_m;          // tile rows (of 128 or of 256 for CTA pairs) per raster group
   int stall_test;
+  int act;              // EpilogueAct
   uint32_t* status;
   // Combining the sparsify pass's K-range partials inside the pair GEMM (instead
   // of finalize_kernel): fin_mode 1 = s and bf16(T / s), 2 = bf16(T) only, 0 =

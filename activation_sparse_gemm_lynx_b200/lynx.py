@@ -24,6 +24,9 @@ LYNX_ERR_WORKSPACE_TOO_SMALL = 4
 LYNX_ERR_CUDA = 5
 LYNX_ERR_DEVICE_TIMEOUT = 6
 
+LYNX_ACT_NONE = 0
+LYNX_ACT_GELU_TANH = 1
+
 
 class LynxError(RuntimeError):
     def __init__(self, status, what=""):
@@ -56,9 +59,11 @@ def library():
             "lynx_sparsify_noalloc": ([p, i64, i64, p, p, p, p], i32),
             "lynx_sparsify_noalloc_max_rows": ([], i64),
             "lynx_linear": ([p, p, p, p, p, i64, i64, i64, i64, i32, p, p, sz, p], i32),
+            "lynx_linear_act": ([p, p, p, p, p, i64, i64, i64, i64, i32, i32, p, p, sz, p], i32),
             "lynx_linear_dense": ([p, p, p, p, p, i64, i64, i64, i64, p, p, sz, p], i32),
             "lynx_linear_host_workspace_bytes": ([i64, i64, i64, i64], sz),
             "lynx_linear_host": ([p, p, p, p, p, i64, i64, i64, i64, i32, p, p, sz, p], i32),
+            "lynx_linear_host_act": ([p, p, p, p, p, i64, i64, i64, i64, i32, i32, p, p, sz, p], i32),
             "lynx_sparse_gemm": ([p, p, p, p, p, p, i64, i64, i64, i64, p, p], i32),
             "lynx_check_error": ([p, p], i32),
             "lynx_meta_hw_to_canonical": ([p, p, i64, i64], i32),
@@ -215,9 +220,7 @@ def _linear_args(X, W, bias, A, B):
     return M, N, K, r
 
 
-def lynx_linear(X, W, bias=None, A=None, B=None, skip_sparsify=False, Y=None, workspace=None,
-                stream=None):
-    """Y = S(X) W^T + bias + (X A^T) B^T (S(X) = X if skip_sparsify). Returns Y."""
+def _linear_buffers(X, W, bias, A, B, Y, workspace):
     import torch
 
     M, N, K, r = _linear_args(X, W, bias, A, B)
@@ -228,10 +231,29 @@ def lynx_linear(X, W, bias=None, A=None, B=None, skip_sparsify=False, Y=None, wo
         workspace = torch.empty(lynx_workspace_bytes(M, N, K, r or 64), dtype=torch.uint8,
                                 device=X.device)
     _need(workspace, "workspace", torch.uint8)
+    return M, N, K, r, Y, workspace
+
+
+def lynx_linear(X, W, bias=None, A=None, B=None, skip_sparsify=False, Y=None, workspace=None,
+                stream=None):
+    """Y = S(X) W^T + bias + (X A^T) B^T (S(X) = X if skip_sparsify). Returns Y."""
+    M, N, K, r, Y, workspace = _linear_buffers(X, W, bias, A, B, Y, workspace)
     st = library().lynx_linear(_ptr(X), _ptr(W), _ptr(bias), _ptr(A), _ptr(B), M, N, K, r,
                                1 if skip_sparsify else 0, _ptr(Y), _ptr(workspace),
                                workspace.numel(), _stream(stream))
     _check(st, "lynx_linear")
+    return Y
+
+
+def lynx_linear_act(X, W, bias=None, A=None, B=None, skip_sparsify=False, act=LYNX_ACT_GELU_TANH,
+                    Y=None, workspace=None, stream=None):
+    """Y = act(S(X) W^T + bias + (X A^T) B^T), the activation applied in the
+    GEMM epilogue (LYNX_ACT_NONE or LYNX_ACT_GELU_TANH). Returns Y."""
+    M, N, K, r, Y, workspace = _linear_buffers(X, W, bias, A, B, Y, workspace)
+    st = library().lynx_linear_act(_ptr(X), _ptr(W), _ptr(bias), _ptr(A), _ptr(B), M, N, K, r,
+                                   1 if skip_sparsify else 0, int(act), _ptr(Y), _ptr(workspace),
+                                   workspace.numel(), _stream(stream))
+    _check(st, "lynx_linear_act")
     return Y
 
 
@@ -245,6 +267,16 @@ def lynx_linear_host(X_host, W, bias=None, A=None, B=None, skip_sparsify=False, 
     tensors (pinned for asynchronous copies); W, bias, A, B are CUDA tensors.
     Returns Y_host, complete once `stream` (default: the current stream) has
     reached this point."""
+    return _linear_host(X_host, W, bias, A, B, skip_sparsify, None, Y_host, workspace, stream)
+
+
+def lynx_linear_host_act(X_host, W, bias=None, A=None, B=None, skip_sparsify=False,
+                         act=LYNX_ACT_GELU_TANH, Y_host=None, workspace=None, stream=None):
+    """lynx_linear_host with the activation of lynx_linear_act."""
+    return _linear_host(X_host, W, bias, A, B, skip_sparsify, int(act), Y_host, workspace, stream)
+
+
+def _linear_host(X_host, W, bias, A, B, skip_sparsify, act, Y_host, workspace, stream):
     import torch
 
     if X_host is None or X_host.is_cuda or X_host.dtype != torch.bfloat16 or not X_host.is_contiguous():
@@ -272,10 +304,16 @@ def lynx_linear_host(X_host, W, bias=None, A=None, B=None, skip_sparsify=False, 
     if workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=W.device)
     _need(workspace, "workspace", torch.uint8)
-    st = library().lynx_linear_host(_ptr(X_host), _ptr(W), _ptr(bias), _ptr(A), _ptr(B), M, N, K, r,
-                                    1 if skip_sparsify else 0, _ptr(Y_host), _ptr(workspace),
-                                    workspace.numel(), _stream(stream))
-    _check(st, "lynx_linear_host")
+    if act is None:
+        st = library().lynx_linear_host(_ptr(X_host), _ptr(W), _ptr(bias), _ptr(A), _ptr(B), M, N, K,
+                                        r, 1 if skip_sparsify else 0, _ptr(Y_host), _ptr(workspace),
+                                        workspace.numel(), _stream(stream))
+        _check(st, "lynx_linear_host")
+    else:
+        st = library().lynx_linear_host_act(_ptr(X_host), _ptr(W), _ptr(bias), _ptr(A), _ptr(B), M, N,
+                                            K, r, 1 if skip_sparsify else 0, act, _ptr(Y_host),
+                                            _ptr(workspace), workspace.numel(), _stream(stream))
+        _check(st, "lynx_linear_host_act")
     return Y_host
 
 

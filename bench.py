@@ -69,6 +69,9 @@ def parse_args(argv=None):
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["lynx", "reference"], default="lynx")
     ap.add_argument("--workload", default="mlp_up")
+    ap.add_argument("--act", choices=["none", "gelu_tanh"], default="none",
+                    help="activation applied in the GEMM epilogue (lynx_linear_act); the "
+                         "comparisons then apply the same activation as a separate pass")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="approximate CPU time of the oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -198,12 +201,14 @@ class ClockSampler:
 # ---------------------------------------------------------------------------
 # the CPU oracle on a bounded sample of the workload
 
-def oracle_sample(inp, rows, skip=False):
+def oracle_sample(inp, rows, skip=False, act="none"):
     import oracle
 
     X = inp["X"][:rows]
     t0 = time.perf_counter()
-    oracle.linear(X, inp["W"], inp["bias"], inp["A"], inp["B"], skip=skip)
+    Y, _, _ = oracle.linear(X, inp["W"], inp["bias"], inp["A"], inp["B"], skip=skip)
+    if act == "gelu_tanh":
+        oracle.gelu_tanh(Y)
     return time.perf_counter() - t0
 
 
@@ -248,9 +253,9 @@ def single_thread_sample(inp, shape, target_s):
             "sample": f"{rows} token rows, {t:.1f} s"}
 
 
-def cpu_baseline(inp, shape, target_s):
+def cpu_baseline(inp, shape, target_s, act="none"):
     rows, cores = calibrate_oracle_rows(inp, target_s, shape.M)
-    t = oracle_sample(inp, rows)
+    t = oracle_sample(inp, rows, act=act)
     flops = 2.0 * rows * shape.N * shape.K
     return {"value": flops / t / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
             "sample": f"{rows} of {shape.M} token rows of {shape.name} (rows are independent), "
@@ -336,14 +341,26 @@ def run_lynx(args):
     Xh = torch.from_numpy(inp["X"].view(np.int16)).view(torch.bfloat16).pin_memory()
     Yh = torch.empty((M, N), dtype=torch.bfloat16).pin_memory()
 
+    act = {"none": lynx.LYNX_ACT_NONE, "gelu_tanh": lynx.LYNX_ACT_GELU_TANH}[args.act]
+
     def step_linear():
-        lynx.lynx_linear(X, W, bias, A, B, Y=Y, workspace=ws)
+        if act == lynx.LYNX_ACT_NONE:
+            lynx.lynx_linear(X, W, bias, A, B, Y=Y, workspace=ws)
+        else:
+            lynx.lynx_linear_act(X, W, bias, A, B, act=act, Y=Y, workspace=ws)
 
     def step_dense_lynx():
-        lynx.lynx_linear(X, W, bias, A, B, skip_sparsify=True, Y=Y, workspace=ws)
+        lynx.lynx_linear_act(X, W, bias, A, B, skip_sparsify=True, act=act, Y=Y, workspace=ws)
 
     def step_dense_torch():
         torch.matmul(X, W.t(), out=Yd)
+        if act != lynx.LYNX_ACT_NONE:
+            torch.nn.functional.gelu(Yd, approximate="tanh")
+
+    def step_unfused_act():
+        # the plain layer, then the activation as a pass of its own over Y
+        lynx.lynx_linear(X, W, bias, A, B, Y=Y, workspace=ws)
+        torch.nn.functional.gelu(Y, approximate="tanh")
 
     ws_host = torch.empty(lynx.lynx_linear_host_workspace_bytes(M, N, K, r), dtype=torch.uint8,
                           device="cuda")
@@ -351,7 +368,10 @@ def run_lynx(args):
     def step_e2e():
         # the C-ABI call on host buffers: copies in, the layer and copies out,
         # pipelined over row chunks inside the library
-        lynx.lynx_linear_host(Xh, W, bias, A, B, Y_host=Yh, workspace=ws_host)
+        if act == lynx.LYNX_ACT_NONE:
+            lynx.lynx_linear_host(Xh, W, bias, A, B, Y_host=Yh, workspace=ws_host)
+        else:
+            lynx.lynx_linear_host_act(Xh, W, bias, A, B, act=act, Y_host=Yh, workspace=ws_host)
 
     def timed(step, n, split=False):
         """Per-step device times (ms) of n steps, L2 flushed before each."""
@@ -429,6 +449,11 @@ def run_lynx(args):
     for _ in range(3):
         step_e2e()
     e2e_ms = max_over_ranks(statistics.mean(timed(step_e2e, ncmp)), world)
+    unfused_ms = None
+    if act != lynx.LYNX_ACT_NONE:
+        for _ in range(3):
+            step_unfused_act()
+        unfused_ms = max_over_ranks(statistics.mean(timed(step_unfused_act, ncmp)), world)
 
     flops = 2.0 * M * N * K
     peaks = load_peaks()
@@ -452,7 +477,9 @@ def run_lynx(args):
         "dtype": "bf16",
         "data": "synthetic (seeded numpy draws rounded to bf16; random weights)",
         "config": {
-            "workload": workload_desc(shape), "M": M, "N": N, "K": K, "r": r,
+            "workload": workload_desc(shape) + ("" if act == lynx.LYNX_ACT_NONE
+                                                else ", GELU(tanh) applied in the GEMM epilogue"),
+            "M": M, "N": N, "K": K, "r": r,
             "l2": "flushed before every step (256 MiB write, outside the timed step)",
             "parallelism": f"dp{world} (independent token-row batches per GPU, no collective)",
         },
@@ -484,8 +511,15 @@ def run_lynx(args):
         "clocks": clock_info,
     }
 
+    if unfused_ms is not None:
+        result["config"]["act"] = args.act
+        result["speedup_vs_unfused_act"] = unfused_ms / ms_step
+        result["breakdown_ms"]["linear_then_separate_act"] = unfused_ms
+        result["breakdown_ms"]["dense_torch_matmul"] = dense_ms
+        result["dense_note"] = "torch.matmul then torch GELU (tanh) as a separate pass"
+
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        result["cpu_baseline"] = cpu_baseline(inp, shape, args.cpu_seconds)
+        result["cpu_baseline"] = cpu_baseline(inp, shape, args.cpu_seconds, act=args.act)
 
     if world > 1:
         import torch.distributed as dist

@@ -162,6 +162,38 @@ LYNX_API int lynx_linear(const void* X, const void* W, const void* bias, const v
                 int64_t M, int64_t N, int64_t K, int64_t r, int skip_sparsify, void* Y,
                 void* workspace, size_t workspace_bytes, void* stream);
 
+/* ---- an activation applied in the GEMM epilogue ------------------------ */
+
+/* Activations lynx_linear_act applies to the finished output row. */
+#define LYNX_ACT_NONE 0
+/* GELU, tanh form (Hendrycks & Gimpel, "Gaussian Error Linear Units"):
+ * gelu(v) = v/2 (1 + tanh(sqrt(2/pi) (v + 0.044715 v^3))), the activation
+ * between a DiT block's MLP up- and down-projections; the down-projection
+ * (MLP.Down, the layer the qingkeai.online article takes as its example in
+ * section 02) reads its output as the activation it sparsifies.  Not on the
+ * RT-Lynx pages themselves, which fuse the sparsification steps so that no
+ * intermediate goes back to memory (same article, section 04); this carries
+ * that to the activation pass before the sparsified layer. */
+#define LYNX_ACT_GELU_TANH 1
+
+/* Y = act(S(X) W^T + bias + (X A^T) B^T): lynx_linear with the activation
+ * applied in fp32 to each finished output value before its one bf16 rounding,
+ * inside the GEMM's epilogue.  Saves the separate activation pass over Y (one
+ * read and one write of M*N*2 bytes) that the layer feeding a sparsified
+ * MLP down-projection otherwise needs.
+ *   act: LYNX_ACT_NONE (then the call is lynx_linear) or LYNX_ACT_GELU_TANH;
+ *   any other value returns LYNX_ERR_INVALID_ARG before anything is launched.
+ *   Every other argument, the workspace and the errors are those of
+ *   lynx_linear.  GELU is evaluated as v * sigmoid(2u), u = sqrt(2/pi)
+ *   (v + 0.044715 v^3) (the same function: (1 + tanh u)/2 = sigmoid(2u)), with
+ *   the hardware base-2 exponential and reciprocal approximations (a few fp32
+ *   ulps; values whose magnitude falls below the fp32 normal range may come
+ *   out as zero). */
+LYNX_API int lynx_linear_act(const void* X, const void* W, const void* bias, const void* A,
+                             const void* B, int64_t M, int64_t N, int64_t K, int64_t r,
+                             int skip_sparsify, int act, void* Y, void* workspace,
+                             size_t workspace_bytes, void* stream);
+
 /* ---- the layer on host-memory activations ------------------------------ */
 
 /* Bytes of the device workspace lynx_linear_host needs: device copies of X and
@@ -184,6 +216,13 @@ LYNX_API int lynx_linear_host(const void* X_host, const void* W, const void* bia
                               const void* B, int64_t M, int64_t N, int64_t K, int64_t r,
                               int skip_sparsify, void* Y_host, void* workspace,
                               size_t workspace_bytes, void* stream);
+
+/* lynx_linear_host with an activation in the GEMM epilogue (lynx_linear_act's
+ * act argument); same workspace and errors. */
+LYNX_API int lynx_linear_host_act(const void* X_host, const void* W, const void* bias, const void* A,
+                                  const void* B, int64_t M, int64_t N, int64_t K, int64_t r,
+                                  int skip_sparsify, int act, void* Y_host, void* workspace,
+                                  size_t workspace_bytes, void* stream);
 
 /* The dense path of a layer that selective layer skipping leaves dense
  * (qingkeai.online article section 03.3): Y = X W^T + bias + (X A^T) B^T.

@@ -113,6 +113,23 @@ def test_linear_host_argument_errors(lib):
     assert call(ws_bytes=need - 1) == lynx.LYNX_ERR_WORKSPACE_TOO_SMALL
 
 
+def test_linear_act_argument_errors(lib):
+    def call(act=lynx.LYNX_ACT_GELU_TANH, X=P, Y=P, ws_bytes=1 << 30):
+        return lib.lynx_linear_act(vp(X), vp(P), None, vp(P), vp(P), 256, 512, 512, 64, 0, act,
+                                   vp(Y), vp(P), ws_bytes, None)
+
+    assert call(act=2) == lynx.LYNX_ERR_INVALID_ARG
+    assert call(act=-1) == lynx.LYNX_ERR_INVALID_ARG
+    assert call(X=None) == lynx.LYNX_ERR_INVALID_ARG
+    assert call(Y=P + 8) == lynx.LYNX_ERR_MISALIGNED
+    need = lynx.lynx_workspace_bytes(256, 512, 512, 64)
+    assert call(ws_bytes=need - 1) == lynx.LYNX_ERR_WORKSPACE_TOO_SMALL
+    # the host form checks the activation too
+    hneed = lynx.lynx_linear_host_workspace_bytes(256, 512, 512, 64)
+    assert lib.lynx_linear_host_act(vp(P), vp(P), None, None, None, 256, 512, 512, 0, 0, 7, vp(P),
+                                    vp(P), hneed, None) == lynx.LYNX_ERR_INVALID_ARG
+
+
 def test_sparse_gemm_argument_errors(lib):
     f = lib.lynx_sparse_gemm
     assert f(vp(P), None, None, vp(P), None, None, 128, 256, 512, 0, vp(P), None) == \
