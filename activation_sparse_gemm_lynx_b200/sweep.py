@@ -2,7 +2,9 @@
 replayed from one CUDA graph.
 
 Each layer is one ``lynx_linear`` call (``skip_sparsify`` for the layers that
-selective layer skipping leaves dense: qingkeai.online article section 03.3).
+selective layer skipping leaves dense: qingkeai.online article section 03.3),
+or ``lynx_linear_act`` for a layer whose output takes an activation (the MLP
+up-projection's GELU) in the GEMM epilogue.
 The calls share one workspace, which is safe because they run in order on one
 stream.  Capturing the whole sequence once and replaying it removes the host
 launch work (argument checks, tensor-map encoding, launches) from every step;
@@ -17,7 +19,8 @@ class LinearSweep:
     """Device-resident inputs, weights and outputs of a list of layers.
 
     ``layers`` holds dicts with the bf16-bit numpy arrays ``X``, ``W``, ``bias``,
-    ``A``, ``B`` (as made by ``workloads.make_linear_inputs``) and ``skip``.
+    ``A``, ``B`` (as made by ``workloads.make_linear_inputs``), ``skip`` and
+    optionally ``act`` (a ``lynx.LYNX_ACT_*`` value, default none).
     """
 
     def __init__(self, layers, device="cuda"):
@@ -32,6 +35,7 @@ class LinearSweep:
             N = t["W"].shape[0]
             t["Y"] = torch.empty((M, N), dtype=torch.bfloat16, device=self.device)
             t["skip"] = bool(layer["skip"])
+            t["act"] = int(layer.get("act", lynx.LYNX_ACT_NONE))
             t["shape"] = (M, K, N)
             self.layers.append(t)
             ws_bytes = max(ws_bytes, lynx.lynx_workspace_bytes(M, N, K, 64))
@@ -54,8 +58,12 @@ class LinearSweep:
     def run(self):
         """Enqueue every layer on the current stream."""
         for t in self.layers:
-            lynx.lynx_linear(t["X"], t["W"], t["bias"], t["A"], t["B"], skip_sparsify=t["skip"],
-                             Y=t["Y"], workspace=self.workspace)
+            if t["act"] == lynx.LYNX_ACT_NONE:
+                lynx.lynx_linear(t["X"], t["W"], t["bias"], t["A"], t["B"], skip_sparsify=t["skip"],
+                                 Y=t["Y"], workspace=self.workspace)
+            else:
+                lynx.lynx_linear_act(t["X"], t["W"], t["bias"], t["A"], t["B"], skip_sparsify=t["skip"],
+                                     act=t["act"], Y=t["Y"], workspace=self.workspace)
 
     def capture(self):
         """Record one pass into a CUDA graph.  Run the sweep once first (the

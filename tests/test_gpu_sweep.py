@@ -97,3 +97,43 @@ def test_full_size_sweep_layer_sampled_rows(layer, skip):
                                  want_sx=True)
     worst, fro = helpers.y_tolerance_check(y, y_ref, sx, helpers.f32(inp["W"]).astype(np.float64))
     assert worst <= 1.0 and fro <= 5e-3, (layer, skip, worst, fro)
+
+
+def test_sweep_with_gelu_on_up_layers():
+    """The sweep with the MLP up-projections' GELU in their GEMM epilogue: the
+    graph replays the eager pass bit for bit, and an up layer matches the
+    oracle's gelu_tanh(linear) within the layer's bar times GELU's largest
+    slope (1.13)."""
+    torch.cuda.set_device(0)
+    plan = workloads.sweep_plan(M=384)[:8]  # two blocks
+    layers = []
+    for (_b, name, M, K, N, kind, skip, seed) in plan:
+        inp = workloads.make_linear_inputs(M, K, N, seed=seed, x_kind=kind)
+        inp["skip"] = skip
+        if name == "up":
+            inp["act"] = lynx.LYNX_ACT_GELU_TANH
+        layers.append(inp)
+    sweep = LinearSweep(layers, device="cuda:0")
+    sweep.run()
+    torch.cuda.synchronize()
+    eager = [t["Y"].clone() for t in sweep.layers]
+    for t in sweep.layers:
+        t["Y"].zero_()
+    sweep.capture()
+    sweep.replay()
+    torch.cuda.synchronize()
+    st, code = lynx.lynx_check_error()
+    assert st == lynx.LYNX_OK, (st, code)
+    for t, e in zip(sweep.layers, eager):
+        assert torch.equal(t["Y"].view(torch.int16), e.view(torch.int16))
+    i = next(i for i, p in enumerate(plan) if p[1] == "up")
+    inp = layers[i]
+    rows = np.array([0, 5, 127, 128, 255, 256, 383])
+    y = helpers.f32(host(sweep.layers[i]["Y"])).astype(np.float64)[rows]
+    y_pre, _, sx = oracle.linear(inp["X"][rows], inp["W"], inp["bias"], inp["A"], inp["B"],
+                                 skip=inp["skip"], want_sx=True)
+    y_ref = oracle.gelu_tanh(y_pre)
+    bound = 1.13 * 2e-2 * np.outer(np.linalg.norm(sx, axis=1),
+                                   np.linalg.norm(helpers.f32(inp["W"]).astype(np.float64), axis=1))
+    assert float((np.abs(y - y_ref) / bound).max()) <= 1.0
+    assert np.linalg.norm(y - y_ref) <= 1.13 * 5e-3 * np.linalg.norm(y_pre)
