@@ -96,10 +96,13 @@ __device__ __forceinline__ uint32_t select_group(uint32_t w0, uint32_t w1, uint3
   la_odd = __fadd_rn(la_odd, fabsf(__uint_as_float(f1)));
   la_even = __fadd_rn(la_even, fabsf(__uint_as_float(f2)));
   la_odd = __fadd_rn(la_odd, fabsf(__uint_as_float(f3)));
-  const uint32_t k0 = (f0 & 0x7FFF0000u) | 3u;
-  const uint32_t k1 = (f1 & 0x7FFF0000u) | 2u;
-  const uint32_t k2 = (f2 & 0x7FFF0000u) | 1u;
-  const uint32_t k3 = f3 & 0x7FFF0000u;
+  // the 15 magnitude bits go to bits 17..31 by a multiply that drops the sign
+  // (the FMA pipe, not the busier ALU pipe); the low 17 bits of each product
+  // are zero, so 3 - i fits below them
+  const uint32_t k0 = w0 * 131072u + 3u;
+  const uint32_t k1 = f1 * 2u + 2u;
+  const uint32_t k2 = w1 * 131072u + 1u;
+  const uint32_t k3 = f3 * 2u;
   const uint32_t p = max(k0, k1), q = min(k0, k1);
   const uint32_t r = max(k2, k3), u = min(k2, k3);
   const uint32_t t1 = max(p, r);
