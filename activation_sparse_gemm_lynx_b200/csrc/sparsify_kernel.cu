@@ -108,11 +108,11 @@ __device__ __forceinline__ uint32_t select_group(uint32_t w0, uint32_t w1, uint3
   const uint32_t t1 = max(p, r);
   const uint32_t t2 = max(min(p, r), max(q, u));
   const uint32_t a = t1 & 3u, b = t2 & 3u;  // 3 - index of the two winners
-  const uint32_t lo = 3u ^ max(a, b);
-  const uint32_t hi = 3u ^ min(a, b);
-  // byte selector picking elements lo and hi out of the 8 bytes (w1:w0)
-  kept = __byte_perm(w0, w1, 0x1010u + lo * 0x22u + hi * 0x2200u);
-  return lo | (hi << 2);
+  const uint32_t mx = max(a, b), mn = min(a, b);  // lo = 3 - mx, hi = 3 - mn
+  // byte selector picking elements lo and hi out of the 8 bytes (w1:w0):
+  // 0x1010 + lo * 0x22 + hi * 0x2200, with the constant parts folded
+  kept = __byte_perm(w0, w1, 0x7676u - mx * 0x22u - mn * 0x2200u);
+  return 15u - mx - mn * 4u;  // lo | hi << 2
 }
 
 __device__ __forceinline__ uint32_t scale_pair(uint32_t w, float s) {
@@ -316,7 +316,7 @@ sparsify_kernel(const __grid_constant__ SparsifyLaunch p) {
       const uint32_t n1 = select_group(v0.z, v0.w, kw[1], la0, la1);
       const uint32_t n2 = select_group(v1.x, v1.y, kw[2], la0, la1);
       const uint32_t n3 = select_group(v1.z, v1.w, kw[3], la0, la1);
-      const uint32_t nib = n0 | (n1 << 4) | (n2 << 8) | (n3 << 12);
+      const uint32_t nib = n0 + n1 * 16u + n2 * 256u + n3 * 4096u;  // disjoint nibbles
       add_abs_pair(lk0, lk1, kw[0]);
       add_abs_pair(lk0, lk1, kw[1]);
       add_abs_pair(lk0, lk1, kw[2]);
