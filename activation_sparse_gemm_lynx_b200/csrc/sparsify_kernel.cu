@@ -295,13 +295,17 @@ sparsify_kernel(const __grid_constant__ SparsifyLaunch p) {
     const uint32_t vst_off = row * 64 + ((qt ^ ((row >> 1) & 3)) << 4);
     // fp32 partial sums of |x| and |kept|, even and odd positions apart
     float la0 = 0.f, la1 = 0.f, lk0 = 0.f, lk1 = 0.f;
-    // this thread's metadata field of box b: block (kabs >> 7) of the row
+    // this thread's metadata field of a box: block (kabs >> 7) of the row
     // block, 16-bit word lane*8 + ((kabs >> 5) & 3)*2 + hsel, kabs = its first
-    // dense column (32-bit: K < 2^30)
-    const uint32_t meta_lane_off = meta_lane * 8 + meta_hsel;
-    uint32_t kabs = static_cast<uint32_t>(kcol0) + 16 * qt;
+    // dense column (32-bit: K < 2^30).  From one box to the next kabs grows by
+    // 64: within a 128-column block (bit 6 of kabs clear) the word index grows
+    // by 4; across a block boundary by 1024 - 4.
+    const uint32_t kabs0 = static_cast<uint32_t>(kcol0) + 16 * qt;
+    uint16_t* meta_ptr = meta_row_blocks + ((kabs0 >> 7) << 10) + meta_lane * 8 + meta_hsel +
+                         (((kabs0 >> 5) & 3u) << 1);
+    uint32_t meta_hi_half = (kabs0 >> 6) & 1u;
     uint32_t slot = 0, phase = 0;
-    for (int b = 0; b < nboxes; ++b, kabs += 64) {
+    for (int b = 0; b < nboxes; ++b) {
       bool ok = !sm.abort_flag;
       if (ok && !mbar_wait(&sm.full[slot], phase)) {
         set_abort(sm, p.status, kDevTimeoutFull);
@@ -321,8 +325,9 @@ sparsify_kernel(const __grid_constant__ SparsifyLaunch p) {
       add_abs_pair(lk0, lk1, kw[1]);
       add_abs_pair(lk0, lk1, kw[2]);
       add_abs_pair(lk0, lk1, kw[3]);
-      meta_row_blocks[((kabs >> 7) << 10) + meta_lane_off + (((kabs >> 5) & 3u) << 1)] =
-          static_cast<uint16_t>(nib);
+      *meta_ptr = static_cast<uint16_t>(nib);
+      meta_ptr += meta_hi_half ? 1020 : 4;
+      meta_hi_half ^= 1u;
       // the store of box b - 2 has read this staging buffer
       if (!mbar_wait(&sm.vfree[b & 1], static_cast<uint32_t>((b >> 1) & 1) ^ 1u)) {
         set_abort(sm, p.status, kDevTimeoutEmpty);
