@@ -289,3 +289,36 @@ def test_device_timeout_in_the_fused_layer():
         lynx.lynx_debug_set_stall(False)
     assert st == lynx.LYNX_ERR_DEVICE_TIMEOUT and code != 0
     check_linear(inp)
+
+
+def check_selection_all_rows(inp, chunk=1024):
+    """lynx_linear in the benchmark's launch configuration, then its workspace on
+    every row: metadata bit-exact, kept values exact copies of X, s within a few
+    fp32 ulps of the oracle's (rows in chunks, to bound host memory)."""
+    X = inp["X"]
+    M, K = X.shape
+    N = inp["W"].shape[0]
+    ws = torch.empty(lynx.lynx_workspace_bytes(M, N, K, 64), dtype=torch.uint8, device=DEV)
+    lynx.lynx_linear(*[dev(inp[k]) for k in ("X", "W", "bias", "A", "B")], workspace=ws)
+    torch.cuda.synchronize()
+    st, code = lynx.lynx_check_error()
+    assert st == lynx.LYNX_OK, (st, code)
+    vals, meta, scale, _ = helpers.workspace_views(ws.cpu().numpy(), M, K)
+    for m0 in range(0, M, chunk):
+        rows = np.arange(m0, min(M, m0 + chunk))
+        ref = oracle.sparsify(X[rows])
+        canon = helpers.canonical_from_hw(meta, M, K, rows)
+        assert np.array_equal(canon, ref["meta"]), f"metadata differs in rows {m0}.."
+        assert np.array_equal(vals[rows], helpers.kept_from_x(X[rows], canon, K)), f"values, rows {m0}.."
+        assert np.allclose(scale[rows], ref["scale"], rtol=4e-6, atol=0), f"s, rows {m0}.."
+
+
+@pytest.mark.parametrize("name", ["attn_out", "mlp_up", "mlp_down"])
+def test_full_size_selection_on_every_row(name):
+    check_selection_all_rows(workloads.make_config_inputs(name))
+
+
+@pytest.mark.parametrize("layer", [0, 3])  # the sweep's qkv (K = 3072) and down (K = 12288) at M = 8192
+def test_sweep_size_selection_on_every_row(layer):
+    _b, _n, M, K, N, kind, _skip, seed = workloads.sweep_plan()[layer]
+    check_selection_all_rows(workloads.make_linear_inputs(M, K, N, seed=seed, x_kind=kind))
