@@ -184,7 +184,8 @@ sparsify_kernel(const __grid_constant__ SparsifyLaunch p) {
   // output, possibly) is read and this call's outputs (possibly still read by
   // it) are written only from here on
   pdl_wait();
-  // finalize_kernel may begin launching; it waits for this whole grid
+  // the next kernel (finalize_kernel, or the GEMM that combines the partials
+  // itself) may begin launching; it waits for this whole grid
   pdl_launch_dependents();
 
   if (warp == 0) {
