@@ -27,9 +27,11 @@
 //               3-stage ring (128-byte swizzle, the UMMA K-major layout)
 //   warp 1      owns TMEM (64 columns), issues tcgen05.mma M=128,N=64,K=16 on
 //               each X tile for the LoRA down-projection
-//   warps 2-17  512 row threads: thread = (row, quarter of each 64-wide tile,
-//               i.e. 16 columns = 4 groups = one 16-bit metadata field); the
-//               kept values of a tile leave through one TMA store.
+//   warps 2-9   256 row threads: thread = (row, half of each 64-wide tile,
+//               i.e. 32 columns = 8 groups = two 16-bit metadata fields); the
+//               kept values of a tile leave through one TMA store.  (Half rows
+//               rather than quarter rows: half the synchronisation per element,
+//               measured slightly faster than twice the threads.)
 //
 // Metadata layout (consumed by tcgen05.cp.128x128b + tcgen05.mma.sp kind::f16,
 // M=128): one 2048-byte block per 128 rows x 128 dense K, 128 TMEM lanes x 16
@@ -49,9 +51,9 @@ namespace lynx {
 namespace {
 
 constexpr int kStages = 3;
-constexpr int kComputeWarps = 16;
-constexpr int kComputeThreads = 32 * kComputeWarps;  // 512
-constexpr int kThreads = 64 + kComputeThreads;        // 576
+constexpr int kComputeWarps = 8;
+constexpr int kComputeThreads = 32 * kComputeWarps;  // 256
+constexpr int kThreads = 64 + kComputeThreads;        // 320
 constexpr uint32_t kXTileBytes = 128 * 64 * 2;        // 16 KB
 constexpr uint32_t kATileBytes = 64 * 64 * 2;         // 8 KB
 constexpr uint32_t kStoreTileBytes = 128 * 32 * 2;    // 8 KB: 128 rows x 32 kept values
@@ -62,7 +64,7 @@ struct __align__(1024) SparsifySmem {
   uint8_t xring[kStages][kXTileBytes];
   uint8_t aring[kStages][kATileBytes];
   uint8_t vstage[2][kStoreTileBytes];  // kept values of one tile, 64-byte swizzle
-  float2 quarter[3][128];              // partial sums of quarters 1..3
+  float2 half1[128];                   // partial sums of the second half of each row
   uint64_t full[kStages];
   uint64_t empty[kStages];     // row threads done with a stage (one arrival per warp)
   uint64_t mma_done[kStages];  // the LoRA MMAs done with a stage (tcgen05.commit)
@@ -281,27 +283,33 @@ sparsify_kernel(const __grid_constant__ SparsifyLaunch p) {
     __syncwarp();
   } else if (do_sel) {
     // ------------------------------------------------------------ row threads
-    const uint32_t qt = (warp - 2) >> 2;      // which 16 columns of each tile
+    const uint32_t hf = (warp - 2) >> 2;      // which 32 columns of each tile
     const uint32_t row = 32 * (warp & 3) + lane;
     const int64_t grow = mb * 128 + row;
-    // metadata: this thread's 16 columns form one 16-bit field of one lane
-    const uint32_t meta_lane = (row & 7) + 8 * (qt & 1) + 16 * (row >> 4);
+    // metadata: this thread's 32 columns form two 16-bit fields, in lanes 8
+    // apart (64 16-bit words) of the same block and word
+    const uint32_t meta_lane = (row & 7) + 16 * (row >> 4);
     const uint32_t meta_hsel = (row >> 3) & 1;
     uint16_t* meta_row_blocks =
         reinterpret_cast<uint16_t*>(p.meta + static_cast<size_t>(mb) * p.kblocks * kMetaBlockBytes);
-    // where this thread's 16 bytes sit in the tile (128-byte swizzle) and its 8
-    // kept values in the 64-byte-swizzled store tile
-    const uint32_t ld_off0 = row * 128 + (((2 * qt) ^ (row & 7)) << 4);
-    const uint32_t ld_off1 = row * 128 + (((2 * qt + 1) ^ (row & 7)) << 4);
-    const uint32_t vst_off = row * 64 + ((qt ^ ((row >> 1) & 3)) << 4);
+    // where this thread's four 16-byte chunks sit in the tile (128-byte
+    // swizzle), and its 16 kept values in the 64-byte-swizzled store tile
+    const uint32_t sw = row & 7;
+    const uint32_t ld_off0 = row * 128 + (((4 * hf + 0) ^ sw) << 4);
+    const uint32_t ld_off1 = row * 128 + (((4 * hf + 1) ^ sw) << 4);
+    const uint32_t ld_off2 = row * 128 + (((4 * hf + 2) ^ sw) << 4);
+    const uint32_t ld_off3 = row * 128 + (((4 * hf + 3) ^ sw) << 4);
+    const uint32_t s64 = (row >> 1) & 3;
+    const uint32_t vst_off0 = row * 64 + (((2 * hf) ^ s64) << 4);
+    const uint32_t vst_off1 = row * 64 + (((2 * hf + 1) ^ s64) << 4);
     // fp32 partial sums of |x| and |kept|, even and odd positions apart
     float la0 = 0.f, la1 = 0.f, lk0 = 0.f, lk1 = 0.f;
-    // this thread's metadata field of a box: block (kabs >> 7) of the row
-    // block, 16-bit word lane*8 + ((kabs >> 5) & 3)*2 + hsel, kabs = its first
-    // dense column (32-bit: K < 2^30).  From one box to the next kabs grows by
-    // 64: within a 128-column block (bit 6 of kabs clear) the word index grows
-    // by 4; across a block boundary by 1024 - 4.
-    const uint32_t kabs0 = static_cast<uint32_t>(kcol0) + 16 * qt;
+    // this thread's first metadata field of a box: block (kabs >> 7) of the
+    // row block, 16-bit word lane*8 + ((kabs >> 5) & 3)*2 + hsel, kabs = its
+    // first dense column (32-bit: K < 2^30).  From one box to the next kabs
+    // grows by 64: within a 128-column block (bit 6 of kabs clear) the word
+    // index grows by 4; across a block boundary by 1024 - 4.
+    const uint32_t kabs0 = static_cast<uint32_t>(kcol0) + 32 * hf;
     uint16_t* meta_ptr = meta_row_blocks + ((kabs0 >> 7) << 10) + meta_lane * 8 + meta_hsel +
                          (((kabs0 >> 5) & 3u) << 1);
     uint32_t meta_hi_half = (kabs0 >> 6) & 1u;
@@ -316,17 +324,21 @@ sparsify_kernel(const __grid_constant__ SparsifyLaunch p) {
       const uint8_t* tile = sm.xring[slot];
       const uint4 v0 = *reinterpret_cast<const uint4*>(tile + ld_off0);
       const uint4 v1 = *reinterpret_cast<const uint4*>(tile + ld_off1);
-      uint32_t kw[4];
+      const uint4 v2 = *reinterpret_cast<const uint4*>(tile + ld_off2);
+      const uint4 v3 = *reinterpret_cast<const uint4*>(tile + ld_off3);
+      uint32_t kw[8];
       const uint32_t n0 = select_group(v0.x, v0.y, kw[0], la0, la1);
       const uint32_t n1 = select_group(v0.z, v0.w, kw[1], la0, la1);
       const uint32_t n2 = select_group(v1.x, v1.y, kw[2], la0, la1);
       const uint32_t n3 = select_group(v1.z, v1.w, kw[3], la0, la1);
-      const uint32_t nib = n0 + n1 * 16u + n2 * 256u + n3 * 4096u;  // disjoint nibbles
-      add_abs_pair(lk0, lk1, kw[0]);
-      add_abs_pair(lk0, lk1, kw[1]);
-      add_abs_pair(lk0, lk1, kw[2]);
-      add_abs_pair(lk0, lk1, kw[3]);
-      *meta_ptr = static_cast<uint16_t>(nib);
+      const uint32_t n4 = select_group(v2.x, v2.y, kw[4], la0, la1);
+      const uint32_t n5 = select_group(v2.z, v2.w, kw[5], la0, la1);
+      const uint32_t n6 = select_group(v3.x, v3.y, kw[6], la0, la1);
+      const uint32_t n7 = select_group(v3.z, v3.w, kw[7], la0, la1);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) add_abs_pair(lk0, lk1, kw[i]);
+      meta_ptr[0] = static_cast<uint16_t>(n0 + n1 * 16u + n2 * 256u + n3 * 4096u);
+      meta_ptr[64] = static_cast<uint16_t>(n4 + n5 * 16u + n6 * 256u + n7 * 4096u);
       meta_ptr += meta_hi_half ? 1020 : 4;
       meta_hi_half ^= 1u;
       // the store of box b - 2 has read this staging buffer
@@ -335,7 +347,8 @@ sparsify_kernel(const __grid_constant__ SparsifyLaunch p) {
         ok = false;
       }
       if (!__all_sync(0xffffffffu, ok)) break;
-      *reinterpret_cast<uint4*>(sm.vstage[b & 1] + vst_off) = make_uint4(kw[0], kw[1], kw[2], kw[3]);
+      *reinterpret_cast<uint4*>(sm.vstage[b & 1] + vst_off0) = make_uint4(kw[0], kw[1], kw[2], kw[3]);
+      *reinterpret_cast<uint4*>(sm.vstage[b & 1] + vst_off1) = make_uint4(kw[4], kw[5], kw[6], kw[7]);
       fence_proxy_async_smem();
       // release the stage only after everything derived from it has been
       // produced: an arrive does not wait for this warp's loads in flight
@@ -348,17 +361,11 @@ sparsify_kernel(const __grid_constant__ SparsifyLaunch p) {
     }
     const float my_la = __fadd_rn(la0, la1);
     const float my_lk = __fadd_rn(lk0, lk1);
-    if (qt > 0) sm.quarter[qt - 1][row] = make_float2(my_la, my_lk);
+    if (hf > 0) sm.half1[row] = make_float2(my_la, my_lk);
     named_bar_sync(kBarCompute, kComputeThreads);
-    if (qt == 0 && grow < p.M) {
-      float a = my_la, k = my_lk;
-#pragma unroll
-      for (int q = 0; q < 3; ++q) {  // fixed order
-        const float2 o = sm.quarter[q][row];
-        a = __fadd_rn(a, o.x);
-        k = __fadd_rn(k, o.y);
-      }
-      p.lpart[static_cast<size_t>(j) * p.M + grow] = make_float2(a, k);
+    if (hf == 0 && grow < p.M) {
+      const float2 o = sm.half1[row];
+      p.lpart[static_cast<size_t>(j) * p.M + grow] = make_float2(__fadd_rn(my_la, o.x), __fadd_rn(my_lk, o.y));
     }
   }
 
