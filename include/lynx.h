@@ -22,7 +22,7 @@
  *     kernels of this library (section 04).
  *
  * Conventions for every entry point:
- *   - Tensors are bf16 (IEEE binary16-brain, 2 bytes), row-major, contiguous,
+ *   - Tensors are bf16 (bfloat16: the upper 16 bits of an IEEE fp32), row-major, contiguous,
  *     given as plain device pointers.  The caller owns and allocates every
  *     buffer; the library never allocates device memory.
  *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
@@ -93,7 +93,8 @@ LYNX_API size_t lynx_vals_bytes(int64_t M, int64_t K);
 LYNX_API size_t lynx_meta_bytes(int64_t M, int64_t K);
 
 /* Bytes of the workspace lynx_linear needs (kept values, metadata, row scales,
- * the bf16 LoRA down-projection [M,64], per-range partial sums, alignment). */
+ * the bf16 LoRA down-projection [M,64], per-range partial sums, one
+ * completion word per GEMM CTA, alignment). */
 LYNX_API size_t lynx_workspace_bytes(int64_t M, int64_t N, int64_t K, int64_t r);
 
 /* ---- the layer --------------------------------------------------------- */
