@@ -99,3 +99,39 @@ def test_weak_scaling_value_counts_all_ranks(world):
     # value = all ranks' dense-equivalent flops / the slowest rank's time
     flops = 2.0 * 4608 * 12288 * 3072
     assert bench.aggregate_tflops(flops, 0.2, world) == pytest.approx(world * flops / 0.2e-3 / 1e12)
+
+
+def test_reference_arm_line_on_rank0(monkeypatch, capsys):
+    """The reference arm (the oracle on the host cores) prints one JSON line with
+    the contract's keys, on the tiny workload."""
+    import json
+
+    import bench
+
+    monkeypatch.setenv("RANK", "0")
+    monkeypatch.setenv("WORLD_SIZE", "1")
+    monkeypatch.setenv("LOCAL_RANK", "0")
+    args = bench.parse_args(["--impl", "reference", "--workload", "tiny", "--steps", "1",
+                             "--warmup", "3"])
+    assert bench.run_reference(args) == 0
+    lines = [ln for ln in capsys.readouterr().out.splitlines() if ln.strip()]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["unit"] == "TFLOP/s" and d["value"] > 0
+    assert d["steps"] == 1 and d["warmup"] == 3 and d["higher_is_better"] is True
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
+    assert d["cpu_baseline"]["cpu"]
+    assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
+    assert d["gpu_launches"] == 0
+
+
+def test_cpu_baseline_reports_cores_model_and_single_thread():
+    import bench
+    from activation_sparse_gemm_lynx_b200 import workloads
+
+    shape = workloads.CONFIGS["tiny"]
+    inp = workloads.make_config_inputs("tiny")
+    b = bench.cpu_baseline(inp, shape, 0.5)
+    assert b["value"] > 0 and b["cores"] >= 1 and b["kind"] == "oracle" and b["cpu"]
+    st = b["single_thread"]
+    assert st["cores"] == 1 and st["value"] > 0
