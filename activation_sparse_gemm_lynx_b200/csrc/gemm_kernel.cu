@@ -96,6 +96,7 @@ lynx_gemm_kernel(const __grid_constant__ GemmLaunch p) {
   const int nk = static_cast<int>(p.K / 64);  // 64 dense K per stage
   const int kblocks = static_cast<int>((p.K + 127) / 128);
   const bool lora = p.lora != 0;
+  const int lsteps = lora ? (p.r + 31) / 32 : 0;  // LoRA-up stages of K = 32 (zero-filled past r)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::kStages; ++s) {
@@ -137,7 +138,7 @@ lynx_gemm_kernel(const __grid_constant__ GemmLaunch p) {
         tile_coords(tile, ntm, ntn, mb, nb);
         const int32_t row0 = mb * 128;
         const int32_t col0 = nb * BN;
-        const int steps = nk + (lora ? 2 : 0);
+        const int steps = nk + lsteps;
         for (int kit = 0; kit < steps; ++kit, ++g) {
           const uint32_t slot = g % C::kStages;
           const uint32_t ph = (g / C::kStages) & 1u;
@@ -199,7 +200,7 @@ lynx_gemm_kernel(const __grid_constant__ GemmLaunch p) {
         }
         tc_fence_after();
         const uint32_t d_tmem = sm.tmem_base + static_cast<uint32_t>(acc * BN);
-        const int steps = nk + (lora ? 2 : 0);
+        const int steps = nk + lsteps;
         uint32_t accumulate = 0;
         for (int kit = 0; kit < steps; ++kit, ++g) {
           const uint32_t slot = g % C::kStages;
@@ -241,8 +242,10 @@ lynx_gemm_kernel(const __grid_constant__ GemmLaunch p) {
               }
             }
           } else {
+            const int l = kit - nk;
 #pragma unroll
             for (int kk = 0; kk < 2; ++kk) {
+              if (32 * l + 16 * kk >= p.r) break;  // past r: the zero-filled half of the box
               const uint64_t da = make_sdesc(sa + 32 * kk, 16, 512, kSw64);
               const uint64_t db = make_sdesc(sb + 32 * kk, 16, 512, kSw64);
               mma_bf16(d_tmem, da, db, idesc_dense, accumulate);
@@ -336,16 +339,13 @@ lynx_gemm_kernel(const __grid_constant__ GemmLaunch p) {
 template <int BN, bool SPARSE>
 cudaError_t launch_variant(const GemmLaunch& p, cudaStream_t stream) {
   const size_t smem = sizeof(GemmSmem<BN, SPARSE>) + 1024;
-  static int configured_device = -1;
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (configured_device != dev) {
-    cudaError_t e = cudaFuncSetAttribute(lynx_gemm_kernel<BN, SPARSE>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem));
-    if (e != cudaSuccess) return e;
-    configured_device = dev;
-  }
+  static std::once_flag once[64];
+  static cudaError_t configured[64];
+  cudaError_t e = once_per_device(once, configured, [smem]() {
+    return cudaFuncSetAttribute(lynx_gemm_kernel<BN, SPARSE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                static_cast<int>(smem));
+  });
+  if (e != cudaSuccess) return e;
   return launch_after_previous(lynx_gemm_kernel<BN, SPARSE>, dim3(static_cast<unsigned>(p.grid)),
                                dim3(kGemmThreads), smem, stream, p);
 }

@@ -83,9 +83,11 @@ struct __align__(1024) PairSmem {
   uint64_t acc_full;           // each CTA's epilogue waits on its own
   uint64_t acc_empty;          // used in the leader CTA (both CTAs' epilogues arrive)
   uint64_t drain;
-  uint64_t fin_done;           // every CTA's rows of s and T are written (fused combining)
+  uint64_t rows_ready;         // the rows of T of all this CTA's tiles are combined (fused, LoRA)
   float bias_s[256];
   uint32_t tmem_base;
+  uint32_t own_claimed[32];    // fused combining: which of the CTA's own slices it claimed
+  int open_slice;              // fused combining: an open slice found in the round of checks
   volatile uint32_t abort_flag;
 };
 
@@ -108,26 +110,44 @@ __device__ __forceinline__ float row_scale_from_partials(const float2* lpart, in
   return (lk == 0.f) ? 1.f : __fdiv_rn(la, lk);
 }
 
-// This CTA's slice of rows: s, and T written as bf16(T / s) (fin_mode 1) or
-// bf16(T) (fin_mode 2), T summed over the K ranges in the fixed order.  256
-// threads, 8 per row, 8 columns of T each.
-__device__ __forceinline__ void finalize_slice(const GemmLaunch& p, uint32_t et) {
-  const int64_t per = (p.M + gridDim.x - 1) / gridDim.x;
-  const int64_t first = static_cast<int64_t>(blockIdx.x) * per;
-  const int64_t last = (first + per < p.M) ? first + per : p.M;
+// tiles walk M first inside a group of `group_m` pair-rows (sized on the host so
+// that the group's A rows stay resident in L2 while W streams once per group)
+__device__ __forceinline__ void pair_tile_coords(int tile, int ntm2, int ntn, int group_m, int& pm,
+                                                 int& nb) {
+  const int per_group = group_m * ntn;
+  const int group = tile / per_group;
+  const int first = group * group_m;
+  const int gm = min(group_m, ntm2 - first);
+  const int in_group = tile - group * per_group;
+  pm = first + in_group % gm;
+  nb = in_group / gm;
+}
+
+// Rows of the sparsify pass's partials are combined in slices of 32 rows: s
+// (fin_mode 1) and, with LoRA, T summed over the K ranges in the fixed order
+// j = 0, 1, ... and written as bf16(T / s) (fin_mode 1) or bf16(T) (fin_mode
+// 2).  256 threads, 8 per row; each takes the row's 8-column chunks sub, sub +
+// 8, ... of r / 8.
+constexpr int kSliceRows = 32;
+constexpr int kMaxOwnSlices = 32;
+
+__device__ __forceinline__ void combine_slice(const GemmLaunch& p, int sl, uint32_t et) {
+  const int64_t row = static_cast<int64_t>(sl) * kSliceRows + (et >> 3);
+  if (row >= p.M) return;
   const uint32_t sub = et & 7u;
-  for (int64_t row = first + (et >> 3); row < last; row += 32) {
-    float s = 1.f;
-    if (p.fin_mode == 1) {
-      s = row_scale_from_partials(p.fin_lpart, p.M, p.fin_split, row);
-      if (sub == 0) p.fin_scale[row] = s;
-    }
+  const int chunks = p.lora ? p.r / 8 : 0;
+  float s = 1.f;
+  if (p.fin_mode == 1) {
+    s = row_scale_from_partials(p.fin_lpart, p.M, p.fin_split, row);
+    if (sub == 0) p.fin_scale[row] = s;
+  }
+  for (int q = static_cast<int>(sub); q < chunks; q += 8) {
     float4 v[kMaxSplit][2];
 #pragma unroll
     for (int j = 0; j < kMaxSplit; ++j) {
       if (j < p.fin_split) {
         const float4* src = reinterpret_cast<const float4*>(
-            p.fin_tpart + (static_cast<size_t>(j) * p.M + row) * kLoraRank + 8 * sub);
+            p.fin_tpart + (static_cast<size_t>(j) * p.M + row) * p.r + 8 * q);
         v[j][0] = __ldcg(src);
         v[j][1] = __ldcg(src + 1);
       }
@@ -159,49 +179,102 @@ __device__ __forceinline__ void finalize_slice(const GemmLaunch& p, uint32_t et)
       __nv_bfloat162 h = __floats2bfloat162_rn(x0, x1);
       pk[e] = *reinterpret_cast<uint32_t*>(&h);
     }
-    *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.fin_t) + row * kLoraRank + 8 * sub) =
+    *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.fin_t) + row * p.r + 8 * q) =
         make_uint4(pk[0], pk[1], pk[2], pk[3]);
   }
 }
 
-// Each CTA publishes the call's epoch in its own word once its slice is
-// written; the words of an earlier call, of an aborted one, or whatever the
-// workspace held hold other values, so they need no reset.  (A single counter
-// updated by compare-and-swap from every CTA serialised them badly.)
-__device__ __forceinline__ void publish_finalized(const GemmLaunch& p) {
-  asm volatile("st.release.gpu.global.u64 [%0], %1;"
-               ::"l"(p.fin_counter + blockIdx.x), "l"(p.fin_epoch) : "memory");
+// After combining a slice: its s and T are read by other CTAs (generic loads)
+// and by TMA (async proxy); thread 0 then publishes the slice as done.
+__device__ __forceinline__ void publish_slices_fence() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+  __threadfence();
 }
 
-// The epilogue threads of each CTA wait (bounded) until every CTA of this call
-// has published its slice: thread i watches word i (and i + 256, ...), so the
-// whole grid is checked in one round of loads; a single acquire fence follows.
-__device__ __forceinline__ bool wait_all_finalized(const GemmLaunch& p, uint32_t et) {
-  const uint64_t t0 = globaltimer_ns();
-  for (uint32_t c = et; c < gridDim.x; c += kEpiThreads) {
-    for (;;) {
-      unsigned long long v;
-      asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p.fin_counter + c) : "memory");
-      if (v == p.fin_epoch) break;
-      if (globaltimer_ns() - t0 > kWaitLimitNs) return false;
-      __nanosleep(64);
+__device__ __forceinline__ void store_release(uint32_t* flag, uint32_t v) {
+  asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(flag), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ uint32_t load_acquire(const uint32_t* flag) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(flag) : "memory");
+  return v;
+}
+
+// Before its first tile, the epilogue warps of a CTA make sure that every row
+// of its tiles is combined.  Each 32-row slice has a state word: 0 open, 1
+// claimed by a CTA that is combining it, 2 done.  First every CTA claims and
+// combines the slices it owns (slice i belongs to CTA i mod grid, so the work
+// is spread evenly); then it checks the slices of its own tiles in one round of
+// acquiring loads, claims and combines any that is still open (its owner has
+// not started), and waits (bounded) only for slices that a running CTA has
+// claimed.  So no CTA waits for one that has not started (the grid needs no
+// co-residency), and the words start at 0 in every call (the sparsify pass of
+// the same call clears them), so neither an earlier call nor a replayed graph
+// can leave a stale "done".  Returns false (in every thread) if a wait ran out.
+template <typename Smem>
+__device__ __noinline__ bool ensure_rows_of_tiles(const GemmLaunch& p, Smem& sm, uint32_t et, int ntm2,
+                                                  int ntn, int first_tile, int tile_step, int ntiles,
+                                                  uint32_t rank) {
+  const int nsl = static_cast<int>((p.M + kSliceRows - 1) / kSliceRows);
+  const int cta = static_cast<int>(blockIdx.x);
+  const int grid = static_cast<int>(gridDim.x);
+  // 1. the slices this CTA owns
+  const int nown = cta < nsl ? min(kMaxOwnSlices, (nsl - cta + grid - 1) / grid) : 0;
+  if (et < static_cast<uint32_t>(nown))
+    sm.own_claimed[et] = atomicCAS(p.fin_flags + cta + static_cast<int>(et) * grid, 0u, 1u) == 0u ? 1u : 0u;
+  named_bar_sync(kBarEpilogue, kEpiThreads);
+  bool any_own = false;
+  for (int k = 0; k < nown; ++k) {
+    if (sm.own_claimed[k]) {
+      combine_slice(p, cta + k * grid, et);
+      any_own = true;
     }
   }
-  asm volatile("fence.acq_rel.gpu;" ::: "memory");
-  return true;
-}
-
-// tiles walk M first inside a group of `group_m` pair-rows (sized on the host so
-// that the group's A rows stay resident in L2 while W streams once per group)
-__device__ __forceinline__ void pair_tile_coords(int tile, int ntm2, int ntn, int group_m, int& pm,
-                                                 int& nb) {
-  const int per_group = group_m * ntn;
-  const int group = tile / per_group;
-  const int first = group * group_m;
-  const int gm = min(group_m, ntm2 - first);
-  const int in_group = tile - group * per_group;
-  pm = first + in_group % gm;
-  nb = in_group / gm;
+  if (any_own) {
+    publish_slices_fence();
+    named_bar_sync(kBarEpilogue, kEpiThreads);
+    if (et < static_cast<uint32_t>(nown) && sm.own_claimed[et])
+      store_release(p.fin_flags + cta + static_cast<int>(et) * grid, 2u);
+  }
+  // 2. the slices of this CTA's tiles: entry e = (tile index e / 4, slice e % 4
+  // of the tile's 128-row block of this CTA)
+  const int mine = first_tile < ntiles ? (ntiles - first_tile + tile_step - 1) / tile_step : 0;
+  const int entries = 4 * mine;
+  const uint64_t t0 = globaltimer_ns();
+  for (;;) {
+    bool pending = false;
+    int open = -1;
+    for (int e = static_cast<int>(et); e < entries; e += kEpiThreads) {
+      int pm, nb;
+      pair_tile_coords(first_tile + (e >> 2) * tile_step, ntm2, ntn, p.group_m, pm, nb);
+      const int sl = (pm * 2 + static_cast<int>(rank)) * 4 + (e & 3);
+      if (sl >= nsl) continue;
+      const uint32_t v = load_acquire(p.fin_flags + sl);
+      if (v != 2u) pending = true;
+      if (v == 0u) open = sl;
+    }
+    if (et == 0) sm.open_slice = -1;
+    named_bar_sync(kBarEpilogue, kEpiThreads);
+    if (open >= 0) atomicMax(&sm.open_slice, open);
+    if (!named_bar_red_or(kBarEpilogue, kEpiThreads, pending)) return true;
+    const int sl = sm.open_slice;
+    if (sl >= 0) {
+      // an open slice: its owner has not got this far; combine it here
+      if (et == 0) sm.own_claimed[0] = atomicCAS(p.fin_flags + sl, 0u, 1u) == 0u ? 1u : 0u;
+      named_bar_sync(kBarEpilogue, kEpiThreads);
+      if (sm.own_claimed[0]) {
+        combine_slice(p, sl, et);
+        publish_slices_fence();
+        named_bar_sync(kBarEpilogue, kEpiThreads);
+        if (et == 0) store_release(p.fin_flags + sl, 2u);
+      }
+    } else {
+      __nanosleep(256);
+    }
+    const bool late = globaltimer_ns() - t0 > kWaitLimitNs;
+    if (named_bar_red_or(kBarEpilogue, kEpiThreads, late)) return false;
+  }
 }
 
 template <bool SPARSE, int ACT>
@@ -224,7 +297,9 @@ lynx_gemm_pair_kernel(const __grid_constant__ GemmLaunch p) {
   const int nk = static_cast<int>(p.K / C::kBK);
   const int kblocks = static_cast<int>((p.K + 127) / 128);
   const bool lora = p.lora != 0;
-  const int steps = nk + (lora ? 2 : 0);
+  const int lsteps = lora ? (p.r + 31) / 32 : 0;  // LoRA-up stages of K = 32 (zero-filled past r)
+  const int steps = nk + lsteps;
+  const bool fused = p.fin_mode != 0;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::kStages; ++s) {
@@ -234,7 +309,7 @@ lynx_gemm_pair_kernel(const __grid_constant__ GemmLaunch p) {
     mbar_init(&sm.acc_full, 1);
     mbar_init(&sm.acc_empty, 2 * 8);
     mbar_init(&sm.drain, 1);
-    mbar_init(&sm.fin_done, 1);
+    mbar_init(&sm.rows_ready, 1);
     sm.abort_flag = 0u;
     fence_mbar_init();
   }
@@ -262,7 +337,7 @@ lynx_gemm_pair_kernel(const __grid_constant__ GemmLaunch p) {
       }
       uint32_t g = 0;
       bool ok = !p.stall_test;
-      bool fin_ready = p.fin_mode == 0;
+      bool rows_ready = !fused;
       for (int tile = cluster_id; ok && tile < ntiles; tile += nclusters) {
         int pm, nb;
         pair_tile_coords(tile, ntm2, ntn, p.group_m, pm, nb);
@@ -300,9 +375,10 @@ lynx_gemm_pair_kernel(const __grid_constant__ GemmLaunch p) {
             }
           } else {
             const int l = kit - nk;
-            if (!fin_ready) {
-              // T of every row is written (by the epilogue warps' round of checks)
-              if (sm.abort_flag || !mbar_wait(&sm.fin_done, 0)) {
+            if (!rows_ready) {
+              // the rows of T of every tile of this CTA are combined (the
+              // epilogue warps saw it)
+              if (sm.abort_flag || !mbar_wait(&sm.rows_ready, 0)) {
                 if (!sm.abort_flag) {
                   record_error(p.status, kDevTimeoutFinalize);
                   sm.abort_flag = 1u;
@@ -310,8 +386,12 @@ lynx_gemm_pair_kernel(const __grid_constant__ GemmLaunch p) {
                 ok = false;
                 break;
               }
+              if (sm.abort_flag) {
+                ok = false;
+                break;
+              }
               asm volatile("fence.proxy.async.global;" ::: "memory");  // T is then read by TMA
-              fin_ready = true;
+              rows_ready = true;
             }
             if (leader) mbar_arrive_expect_tx(&sm.full[slot], 2u * (C::kLoraABytes + C::kLoraBBytes));
             tma_load_2d_pair(st, &p.tm_t, lead_full, l * 32, row0);
@@ -389,8 +469,10 @@ lynx_gemm_pair_kernel(const __grid_constant__ GemmLaunch p) {
               }
             }
           } else {
+            const int l = kit - nk;
 #pragma unroll
             for (int kk = 0; kk < 2; ++kk) {
+              if (32 * l + 16 * kk >= p.r) break;  // past r: the zero-filled half of the box
               const uint64_t da = make_sdesc(sa + 32 * kk, 16, 512, kSw64);
               const uint64_t db = make_sdesc(sb + 32 * kk, 16, 512, kSw64);
               if (elect_one()) mma_bf16_pair(d_tmem, da, db, idesc_dense, accumulate);
@@ -444,22 +526,15 @@ lynx_gemm_pair_kernel(const __grid_constant__ GemmLaunch p) {
     const uint32_t et = threadIdx.x - 64u;     // 0..255
     const __nv_bfloat16* bias = static_cast<const __nv_bfloat16*>(p.bias);
     const uint32_t lead_acc_empty = mapa_shared(smem_u32(&sm.acc_empty), 0);
-    if (p.fin_mode != 0) {
-      // before the first accumulator is ready: this CTA's rows of s and T
-      finalize_slice(p, et);
-      __threadfence();
-      named_bar_sync(kBarEpilogue, kEpiThreads);
-      if (et == 0) publish_finalized(p);
-      // then every other CTA's slice: the producer loads T once this is done
-      const bool all = wait_all_finalized(p, et);
-      if (named_bar_red_or(kBarEpilogue, kEpiThreads, !all)) {
-        if (et == 0 && !sm.abort_flag) {
-          record_error(p.status, kDevTimeoutFinalize);
-          sm.abort_flag = 1u;
-        }
-      } else if (et == 0) {
-        mbar_arrive(&sm.fin_done);
+    if (fused) {
+      // s and T of this CTA's 128 rows of each of its tiles, each 32-row slice
+      // combined once per call
+      const bool rows_ok = ensure_rows_of_tiles(p, sm, et, ntm2, ntn, cluster_id, nclusters, ntiles, rank);
+      if (et == 0 && !rows_ok && !sm.abort_flag) {
+        record_error(p.status, kDevTimeoutFinalize);
+        sm.abort_flag = 1u;
       }
+      if (et == 0 && lora) mbar_arrive(&sm.rows_ready);  // the producer may load T
     }
     int acc_count = 0;
     for (int tile = cluster_id; tile < ntiles; tile += nclusters, ++acc_count) {
@@ -473,8 +548,8 @@ lynx_gemm_pair_kernel(const __grid_constant__ GemmLaunch p) {
         const int64_t n = n_base + et;
         sm.bias_s[et] = (bias != nullptr && n < p.N) ? __bfloat162float(bias[n]) : 0.f;
       }
-      // s of the row: with the fused combining step, written by the slice's
-      // owner before this thread's round of checks (read past L1)
+      // s of the row: with the fused combining step, written by the row block's
+      // owner before the checks above (read past L1)
       float s = 1.f;
       if (row_ok) {
         if (p.fin_mode == 1) s = __ldcg(p.fin_scale + grow);
@@ -544,24 +619,22 @@ lynx_gemm_pair_kernel(const __grid_constant__ GemmLaunch p) {
 }
 
 template <bool SPARSE, int ACT>
-cudaError_t launch_pair_variant(const GemmLaunch& p, cudaStream_t stream) {
-  const size_t smem = sizeof(PairSmem<SPARSE>) + 1024;
-  static int configured_device = -1;
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (configured_device != dev) {
-    cudaError_t e = cudaFuncSetAttribute(lynx_gemm_pair_kernel<SPARSE, ACT>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem));
-    if (e != cudaSuccess) return e;
-    configured_device = dev;
-  }
+cudaError_t configure_pair_variant() {
+  static std::once_flag once[64];
+  static cudaError_t configured[64];
+  return once_per_device(once, configured, []() {
+    return cudaFuncSetAttribute(lynx_gemm_pair_kernel<SPARSE, ACT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                static_cast<int>(sizeof(PairSmem<SPARSE>) + 1024));
+  });
+}
+
+template <bool SPARSE, int ACT>
+cudaLaunchConfig_t pair_config(int grid, cudaStream_t stream, cudaLaunchAttribute (&attr)[2]) {
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(p.grid), 1, 1);
+  cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
   cfg.blockDim = dim3(kThreads, 1, 1);
-  cfg.dynamicSmemBytes = smem;
+  cfg.dynamicSmemBytes = sizeof(PairSmem<SPARSE>) + 1024;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
   attr[0].val.clusterDim.y = 1;
@@ -570,10 +643,46 @@ cudaError_t launch_pair_variant(const GemmLaunch& p, cudaStream_t stream) {
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
+  return cfg;
+}
+
+template <bool SPARSE, int ACT>
+cudaError_t launch_pair_variant(const GemmLaunch& p, cudaStream_t stream) {
+  cudaError_t e = configure_pair_variant<SPARSE, ACT>();
+  if (e != cudaSuccess) return e;
+  cudaLaunchAttribute attr[2];
+  cudaLaunchConfig_t cfg = pair_config<SPARSE, ACT>(p.grid, stream, attr);
   return cudaLaunchKernelEx(&cfg, lynx_gemm_pair_kernel<SPARSE, ACT>, p);
 }
 
+template <bool SPARSE, int ACT>
+int pair_max_clusters_variant() {
+  static std::once_flag once[64];
+  static int clusters[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+  std::call_once(once[dev], [dev]() {
+    clusters[dev] = 0;
+    if (configure_pair_variant<SPARSE, ACT>() != cudaSuccess) return;
+    cudaLaunchAttribute attr[2];
+    cudaLaunchConfig_t cfg = pair_config<SPARSE, ACT>(2, nullptr, attr);
+    cfg.numAttrs = 1;  // the cluster shape is what matters here
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, lynx_gemm_pair_kernel<SPARSE, ACT>, &cfg) == cudaSuccess)
+      clusters[dev] = n;
+    else
+      (void)cudaGetLastError();  // a failed query is not sticky; the caller falls back
+  });
+  return clusters[dev];
+}
+
 }  // namespace
+
+int gemm_pair_max_clusters(bool sparse, int act) {
+  if (act == kActGeluTanh)
+    return sparse ? pair_max_clusters_variant<true, kActGeluTanh>() : pair_max_clusters_variant<false, kActGeluTanh>();
+  return sparse ? pair_max_clusters_variant<true, kActNone>() : pair_max_clusters_variant<false, kActNone>();
+}
 
 cudaError_t launch_gemm_pair(const GemmLaunch& p, cudaStream_t stream) {
   if (p.act == kActGeluTanh)

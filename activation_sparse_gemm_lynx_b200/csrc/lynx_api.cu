@@ -6,13 +6,16 @@
 #include <atomic>
 #include <cstring>
 #include <mutex>
-#include <random>
+#include <unordered_map>
 
 #include "lynx.h"
 #include "lynx_internal.h"
 
-// Per-device status word: the first error code a kernel records wins.
-static __device__ uint32_t g_lynx_status_word;
+// Status words, one per stream: the first error code a kernel launched on the
+// stream records wins.  Slot 0 is shared by the streams that find every other
+// slot taken.
+constexpr int kStatusSlots = 1024;
+static __device__ uint32_t g_lynx_status_words[kStatusSlots];
 
 // Scratch of lynx_sparsify_noalloc: per-split partial row sums, then s (when
 // the caller gives no row_scale buffer).  Sized for LYNX_SPARSIFY_NOALLOC_MAX_ROWS.
@@ -28,17 +31,45 @@ constexpr int kMaxDevices = 64;
 
 std::atomic<int> g_stall{0};
 std::atomic<void*> g_split_event{nullptr};
+std::atomic<int> g_profile_part{0};
 
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 std::once_flag g_encode_once;
 
 struct DeviceState {
   std::once_flag once;
-  uint32_t* status = nullptr;
+  uint32_t* status = nullptr;  // device address of the status word array
   int sms = 0;
   cudaError_t err = cudaSuccess;
+  std::mutex slots_mu;         // guards slot_of and next_slot
+  std::unordered_map<uintptr_t, int> slot_of;
+  int next_slot = 1;
 };
 DeviceState g_dev[kMaxDevices];
+
+// Status word of `stream` (assigned on first use; slot 0 once all are taken).
+// Kernels record their errors there and lynx_check_error(stream) reads it.
+uint32_t* stream_status(DeviceState* ds, cudaStream_t stream) {
+  std::lock_guard<std::mutex> lock(ds->slots_mu);
+  const uintptr_t key = reinterpret_cast<uintptr_t>(stream);
+  auto it = ds->slot_of.find(key);
+  int slot = 0;
+  if (it != ds->slot_of.end()) {
+    slot = it->second;
+  } else if (ds->next_slot < kStatusSlots) {
+    slot = ds->next_slot++;
+    ds->slot_of.emplace(key, slot);
+  }
+  return ds->status + slot;
+}
+
+// The slot of `stream` if it has one (-1 if nothing was ever launched on it).
+int find_stream_slot(DeviceState* ds, cudaStream_t stream) {
+  std::lock_guard<std::mutex> lock(ds->slots_mu);
+  auto it = ds->slot_of.find(reinterpret_cast<uintptr_t>(stream));
+  if (it != ds->slot_of.end()) return it->second;
+  return ds->next_slot >= kStatusSlots ? 0 : -1;
+}
 
 // Streams and events of lynx_linear_host, made once per device: copies in and
 // copies out run on their own streams so that they overlap each other (the link
@@ -103,7 +134,7 @@ DeviceState* device_state() {
   DeviceState& d = g_dev[dev];
   std::call_once(d.once, [&d, dev]() {
     void* p = nullptr;
-    d.err = cudaGetSymbolAddress(&p, g_lynx_status_word);
+    d.err = cudaGetSymbolAddress(&p, g_lynx_status_words);
     if (d.err == cudaSuccess) d.status = static_cast<uint32_t*>(p);
     if (d.err == cudaSuccess) d.err = cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev);
   });
@@ -134,27 +165,24 @@ inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 
 
 inline size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
-// The pair GEMM's grid (at most the SM count) must fit the completion words of
-// its fused partial-combining step in the workspace.
-constexpr int kMaxGemmCtas = 1024;
-
 struct WorkspaceLayout {
-  size_t vals, meta, scale, t, lpart, tpart, counter, total;
+  size_t vals, meta, scale, t, lpart, tpart, flags, total;
 };
 
-// lynx_linear's workspace: kept values | metadata | s | T (or T/s) | partials
+// lynx_linear's workspace: kept values | metadata | s | T (or T/s) | partials |
+// one state word per 32-row slice (the GEMM's combining step)
 WorkspaceLayout workspace_layout(int64_t M, int64_t K, int64_t r) {
-  (void)r;
   const size_t m = static_cast<size_t>(M);
+  const size_t rr = static_cast<size_t>(r > 0 ? r : kLoraRankDefault);
   WorkspaceLayout w;
   w.vals = 0;
   w.meta = align256(w.vals + m * static_cast<size_t>(K));
   w.scale = align256(w.meta + lynx_meta_bytes(M, K));
   w.t = align256(w.scale + m * 4);
-  w.lpart = align256(w.t + m * kLoraRank * 2);
+  w.lpart = align256(w.t + m * rr * 2);
   w.tpart = align256(w.lpart + static_cast<size_t>(kMaxSplit) * m * 8);
-  w.counter = align256(w.tpart + static_cast<size_t>(kMaxSplit) * m * kLoraRank * 4);
-  w.total = align256(w.counter + static_cast<size_t>(kMaxGemmCtas) * 8);  // one word per GEMM CTA
+  w.flags = align256(w.tpart + static_cast<size_t>(kMaxSplit) * m * rr * 4);
+  w.total = align256(w.flags + static_cast<size_t>(fin_slices(M)) * 4);
   return w;
 }
 
@@ -181,10 +209,16 @@ lynx_status check_shape(int64_t M, int64_t N, int64_t K) {
   return LYNX_OK;
 }
 
+bool rank_supported(int64_t r) {
+  return r >= kLoraRankAlign && r <= kLoraRankMax && r % kLoraRankAlign == 0;
+}
+
+// A and B both given (then r is their rank) or both NULL (then r is 0 or any
+// supported rank, which only sizes nothing)
 lynx_status check_lora(const void* A, const void* B, int64_t r) {
   if ((A == nullptr) != (B == nullptr)) return LYNX_ERR_INVALID_ARG;
-  if (A != nullptr && r != kLoraRank) return LYNX_ERR_UNSUPPORTED_SHAPE;
-  if (A == nullptr && r != 0 && r != kLoraRank) return LYNX_ERR_UNSUPPORTED_SHAPE;
+  if (A != nullptr && !rank_supported(r)) return LYNX_ERR_UNSUPPORTED_SHAPE;
+  if (A == nullptr && r != 0 && !rank_supported(r)) return LYNX_ERR_UNSUPPORTED_SHAPE;
   return LYNX_OK;
 }
 
@@ -192,41 +226,27 @@ lynx_status map_cuda(cudaError_t e) { return e == cudaSuccess ? LYNX_OK : LYNX_E
 
 int gemm_bn(int64_t N) { return N >= 1024 ? 256 : 128; }
 
-// Call tags of the fused partial-combining step: unique within the process
-// (48-bit, from a random start), so a completion word left by an earlier call,
-// an aborted one or unrelated data is never taken for this call's.
-std::atomic<unsigned long long> g_epoch{0};
-std::once_flag g_epoch_once;
-
-unsigned long long next_epoch() {
-  std::call_once(g_epoch_once, []() {
-    std::random_device rd;
-    const unsigned long long seed = (static_cast<unsigned long long>(rd()) << 32) ^ rd();
-    g_epoch.store(seed & ((1ull << 47) - 1));
-  });
-  return g_epoch.fetch_add(1) & ((1ull << 48) - 1);
-}
-
 // The pair GEMM combines the sparsify pass's partials itself (no finalize_kernel).
 struct FusedFinalize {
-  int mode = 0;  // 1: s and bf16(T / s); 2: bf16(T)
+  int mode = 0;  // 1: s and (with LoRA) bf16(T / s); 2: bf16(T)
   int split = 1;
   const float2* lpart = nullptr;
   const float* tpart = nullptr;
   float* scale = nullptr;
   void* t = nullptr;
-  unsigned long long* counter = nullptr;
+  uint32_t* flags = nullptr;  // one state word per 32-row slice
 };
 
 lynx_status run_sparsify(DeviceState* ds, const void* X, const void* A, int64_t M, int64_t K,
-                         void* vals, void* meta, float* row_scale, void* t_out, float2* lpart,
-                         float* tpart, int mode, cudaStream_t stream, bool skip_finalize = false) {
+                         int64_t r, void* vals, void* meta, float* row_scale, void* t_out,
+                         float2* lpart, float* tpart, int mode, cudaStream_t stream,
+                         const FusedFinalize* fin = nullptr) {
   SparsifyLaunch p;
   std::memset(&p, 0, sizeof(p));
   if (!encode_bf16_2d(&p.tm_x, X, K, M, K * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B))
     return LYNX_ERR_CUDA;
   if (mode & kModeLora) {
-    if (!encode_bf16_2d(&p.tm_a, A, K, kLoraRank, K * 2, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B))
+    if (!encode_bf16_2d(&p.tm_a, A, K, r, K * 2, 64, static_cast<uint32_t>(r), CU_TENSOR_MAP_SWIZZLE_128B))
       return LYNX_ERR_CUDA;
   }
   if (mode & kModeSelect) {
@@ -242,13 +262,18 @@ lynx_status run_sparsify(DeviceState* ds, const void* X, const void* A, int64_t 
   p.tpart = tpart;
   p.M = M;
   p.K = K;
+  p.r = static_cast<int>((mode & kModeLora) ? r : 0);
   p.mode = mode;
   p.split = choose_sparsify_split(M, K, ds->sms);
   p.boxes_per_cta = static_cast<int>(K / 64 / p.split);
   p.kblocks = static_cast<int>((K + 127) / 128);
   p.stall_test = g_stall.load();
-  p.skip_finalize = skip_finalize ? 1 : 0;
-  p.status = ds->status;
+  p.skip_finalize = fin != nullptr ? 1 : 0;
+  if (fin != nullptr) {
+    p.fin_flags = fin->flags;
+    p.fin_nflags = static_cast<int>(fin_slices(M));
+  }
+  p.status = stream_status(ds, stream);
   return map_cuda(launch_sparsify(p, stream));
 }
 
@@ -260,8 +285,8 @@ bool use_pair_kernel(int64_t M, int64_t N, int64_t K) {
 
 lynx_status run_gemm(DeviceState* ds, const void* a_src, bool sparse, const void* meta,
                      const float* row_scale, const void* T, const void* W, const void* bias,
-                     const void* B, int64_t M, int64_t N, int64_t K, void* Y, cudaStream_t stream,
-                     const FusedFinalize* fin = nullptr, int act = kActNone) {
+                     const void* B, int64_t M, int64_t N, int64_t K, int64_t r, void* Y,
+                     cudaStream_t stream, const FusedFinalize* fin = nullptr, int act = kActNone) {
   GemmLaunch p;
   std::memset(&p, 0, sizeof(p));
   const bool pair = use_pair_kernel(M, N, K);
@@ -285,9 +310,11 @@ lynx_status run_gemm(DeviceState* ds, const void* a_src, bool sparse, const void
     return LYNX_ERR_CUDA;
   const bool lora = (T != nullptr && B != nullptr);
   if (lora) {
-    if (!encode_bf16_2d(&p.tm_t, T, kLoraRank, M, kLoraRank * 2, 32, 128, CU_TENSOR_MAP_SWIZZLE_64B))
+    // boxes of 32 columns; for r % 32 == 16 the last box reads past r, which
+    // the TMA fills with zeros (and the kernels skip that half's MMA)
+    if (!encode_bf16_2d(&p.tm_t, T, r, M, r * 2, 32, 128, CU_TENSOR_MAP_SWIZZLE_64B))
       return LYNX_ERR_CUDA;
-    if (!encode_bf16_2d(&p.tm_lb, B, kLoraRank, N, kLoraRank * 2, 32, b_rows, CU_TENSOR_MAP_SWIZZLE_64B))
+    if (!encode_bf16_2d(&p.tm_lb, B, r, N, r * 2, 32, b_rows, CU_TENSOR_MAP_SWIZZLE_64B))
       return LYNX_ERR_CUDA;
   }
   if (pair && !encode_bf16_2d(&p.tm_y, Y, N, M, N * 2, 16, 32, CU_TENSOR_MAP_SWIZZLE_32B))
@@ -299,16 +326,20 @@ lynx_status run_gemm(DeviceState* ds, const void* a_src, bool sparse, const void
   p.M = M;
   p.N = N;
   p.K = K;
+  p.r = lora ? static_cast<int>(r) : 0;
   p.sparse = sparse ? 1 : 0;
   p.lora = lora ? 1 : 0;
   p.bn = bn;
   p.stall_test = g_stall.load();
   p.act = act;
-  p.status = ds->status;
+  p.status = stream_status(ds, stream);
   if (pair) {
     const int64_t ntm2 = (M + 255) / 256;
     const int64_t tiles = ntm2 * ((N + 255) / 256);
-    const int64_t pairs = ds->sms / 2;
+    // one CTA pair per TPC, no more pairs than the device can hold at once
+    int64_t pairs = ds->sms / 2;
+    const int fit = gemm_pair_max_clusters(sparse, act);
+    if (fit > 0 && fit < pairs) pairs = fit;
     p.grid = static_cast<int>(2 * (tiles < pairs ? tiles : pairs));
     // raster group: as many 256-row pair-rows of A as fit in ~40 MB of L2, so
     // the group's A stays resident while W streams once per group
@@ -323,8 +354,7 @@ lynx_status run_gemm(DeviceState* ds, const void* a_src, bool sparse, const void
       p.fin_tpart = fin->tpart;
       p.fin_scale = fin->scale;
       p.fin_t = fin->t;
-      p.fin_counter = fin->counter;
-      p.fin_epoch = next_epoch();
+      p.fin_flags = fin->flags;
     }
     return map_cuda(launch_gemm_pair(p, stream));
   }
@@ -391,7 +421,9 @@ const char* lynx_status_string(int status) {
 
 int lynx_version(void) { return (1 << 16) | 0; }
 
-int lynx_lora_rank(void) { return kLoraRank; }
+int lynx_lora_rank(void) { return kLoraRankDefault; }
+
+int lynx_lora_rank_supported(int64_t r) { return rank_supported(r) ? 1 : 0; }
 
 size_t lynx_vals_bytes(int64_t M, int64_t K) {
   if (M < 0 || K < 0) return 0;
@@ -430,7 +462,7 @@ int lynx_sparsify(const void* X, int64_t M, int64_t K, void* vals, void* meta, f
   if (ds == nullptr) return LYNX_ERR_CUDA;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   float* scale = row_scale ? row_scale : reinterpret_cast<float*>(ws + wl.scale);
-  return run_sparsify(ds, X, nullptr, M, K, vals, meta, scale, nullptr,
+  return run_sparsify(ds, X, nullptr, M, K, 0, vals, meta, scale, nullptr,
                       reinterpret_cast<float2*>(ws + wl.lpart), nullptr, kModeSelect | kModeScaled,
                       static_cast<cudaStream_t>(stream));
 }
@@ -452,7 +484,7 @@ int lynx_sparsify_noalloc(const void* X, int64_t M, int64_t K, void* vals, void*
   uint8_t* scratch = noalloc_scratch();
   if (scratch == nullptr) return LYNX_ERR_CUDA;
   float* scale = row_scale ? row_scale : reinterpret_cast<float*>(scratch + kNoAllocLpartBytes);
-  return run_sparsify(ds, X, nullptr, M, K, vals, meta, scale, nullptr,
+  return run_sparsify(ds, X, nullptr, M, K, 0, vals, meta, scale, nullptr,
                       reinterpret_cast<float2*>(scratch), nullptr, kModeSelect | kModeScaled,
                       static_cast<cudaStream_t>(stream));
 }
@@ -487,7 +519,7 @@ int lynx_linear_act(const void* X, const void* W, const void* bias, const void* 
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   void* t_buf = lora ? ws + wl.t : nullptr;
   // with the CTA-pair GEMM, the GEMM itself combines the pass's K-range partials
-  const bool fused = use_pair_kernel(M, N, K) && (!skip_sparsify || lora) && ds->sms <= kMaxGemmCtas;
+  const bool fused = use_pair_kernel(M, N, K) && (!skip_sparsify || lora);
   FusedFinalize fin;
   if (fused) {
     fin.mode = skip_sparsify ? 2 : 1;
@@ -495,29 +527,40 @@ int lynx_linear_act(const void* X, const void* W, const void* bias, const void* 
     fin.lpart = reinterpret_cast<const float2*>(ws + wl.lpart);
     fin.tpart = reinterpret_cast<const float*>(ws + wl.tpart);
     fin.scale = reinterpret_cast<float*>(ws + wl.scale);
-    fin.t = t_buf != nullptr ? t_buf : ws + wl.t;
-    fin.counter = reinterpret_cast<unsigned long long*>(ws + wl.counter);
+    fin.t = t_buf;
+    fin.flags = reinterpret_cast<uint32_t*>(ws + wl.flags);
   }
+  const int part = g_profile_part.load();
   if (!skip_sparsify) {
-    st = run_sparsify(ds, X, A, M, K, ws + wl.vals, ws + wl.meta,
-                      reinterpret_cast<float*>(ws + wl.scale), t_buf,
-                      reinterpret_cast<float2*>(ws + wl.lpart), reinterpret_cast<float*>(ws + wl.tpart),
-                      kModeSelect | (lora ? kModeLora : 0), s, fused);
-    if (st != LYNX_OK) return st;
+    if (part != 2) {
+      st = run_sparsify(ds, X, A, M, K, r, ws + wl.vals, ws + wl.meta,
+                        reinterpret_cast<float*>(ws + wl.scale), t_buf,
+                        reinterpret_cast<float2*>(ws + wl.lpart), reinterpret_cast<float*>(ws + wl.tpart),
+                        kModeSelect | (lora ? kModeLora : 0), s, fused ? &fin : nullptr);
+      if (st != LYNX_OK || part == 1) return st;
+    } else if (fused && cudaMemsetAsync(fin.flags, 0, fin_slices(M) * 4, s) != cudaSuccess) {
+      return LYNX_ERR_CUDA;
+    }
     if (void* ev = g_split_event.load())
       if (cudaEventRecord(static_cast<cudaEvent_t>(ev), s) != cudaSuccess) return LYNX_ERR_CUDA;
     return run_gemm(ds, ws + wl.vals, true, ws + wl.meta, reinterpret_cast<const float*>(ws + wl.scale),
-                    t_buf, W, bias, B, M, N, K, Y, s, fused ? &fin : nullptr, act);
+                    t_buf, W, bias, B, M, N, K, r, Y, s, fused ? &fin : nullptr, act);
   }
   if (lora) {
-    st = run_sparsify(ds, X, A, M, K, nullptr, nullptr, nullptr, t_buf, nullptr,
-                      reinterpret_cast<float*>(ws + wl.tpart), kModeLora, s, fused);
-    if (st != LYNX_OK) return st;
+    if (part != 2) {
+      st = run_sparsify(ds, X, A, M, K, r, nullptr, nullptr, nullptr, t_buf, nullptr,
+                        reinterpret_cast<float*>(ws + wl.tpart), kModeLora, s, fused ? &fin : nullptr);
+      if (st != LYNX_OK || part == 1) return st;
+    } else if (fused && cudaMemsetAsync(fin.flags, 0, fin_slices(M) * 4, s) != cudaSuccess) {
+      return LYNX_ERR_CUDA;
+    }
+  } else if (part == 1) {
+    return LYNX_OK;
   }
   if (void* ev = g_split_event.load())
     if (cudaEventRecord(static_cast<cudaEvent_t>(ev), s) != cudaSuccess) return LYNX_ERR_CUDA;
-  return run_gemm(ds, X, false, nullptr, nullptr, t_buf, W, bias, B, M, N, K, Y, s, fused ? &fin : nullptr,
-                  act);
+  return run_gemm(ds, X, false, nullptr, nullptr, t_buf, W, bias, B, M, N, K, r, Y, s,
+                  fused ? &fin : nullptr, act);
 }
 
 size_t lynx_linear_host_workspace_bytes(int64_t M, int64_t N, int64_t K, int64_t r) {
@@ -605,7 +648,7 @@ int lynx_sparse_gemm(const void* vals, const void* meta, const void* T, const vo
     return LYNX_ERR_MISALIGNED;
   DeviceState* ds = device_state();
   if (ds == nullptr) return LYNX_ERR_CUDA;
-  return run_gemm(ds, vals, true, meta, nullptr, T, W, bias, B, M, N, K, Y,
+  return run_gemm(ds, vals, true, meta, nullptr, T, W, bias, B, M, N, K, r, Y,
                   static_cast<cudaStream_t>(stream));
 }
 
@@ -616,13 +659,15 @@ int lynx_check_error(void* stream, uint32_t* device_code) {
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   cudaError_t e = cudaStreamSynchronize(s);
   if (e != cudaSuccess) return LYNX_ERR_CUDA;
+  const int slot = find_stream_slot(ds, s);
+  if (slot < 0) return LYNX_OK;  // nothing of this library was launched on the stream
+  uint32_t* word = ds->status + slot;
   uint32_t code = 0;
-  e = cudaMemcpyFromSymbolAsync(&code, g_lynx_status_word, sizeof(code), 0, cudaMemcpyDeviceToHost, s);
+  e = cudaMemcpyAsync(&code, word, sizeof(code), cudaMemcpyDeviceToHost, s);
   if (e == cudaSuccess) e = cudaStreamSynchronize(s);
   if (e != cudaSuccess) return LYNX_ERR_CUDA;
   if (code != 0) {
-    const uint32_t zero = 0;
-    e = cudaMemcpyToSymbolAsync(g_lynx_status_word, &zero, sizeof(zero), 0, cudaMemcpyHostToDevice, s);
+    e = cudaMemsetAsync(word, 0, sizeof(uint32_t), s);
     if (e == cudaSuccess) e = cudaStreamSynchronize(s);
     if (e != cudaSuccess) return LYNX_ERR_CUDA;
   }
@@ -688,5 +733,10 @@ int lynx_meta_canonical_to_hw(const uint8_t* canonical, uint8_t* hw, int64_t M, 
 int lynx_debug_set_stall(int enable) { return g_stall.exchange(enable ? 1 : 0); }
 
 void* lynx_profile_set_split_event(void* event) { return g_split_event.exchange(event); }
+
+int lynx_profile_set_part(int part) {
+  if (part < 0 || part > 2) return -1;
+  return g_profile_part.exchange(part);
+}
 
 }  // extern "C"

@@ -23,10 +23,11 @@
 //   rescale_kernel   standalone S(X): kept values v -> bf16(v * s).
 //
 // sparsify_kernel, per CTA (2 CTAs per SM):
-//   warp 0      TMA producer: 128x64 tiles of X (and 64x64 tiles of A) into a
+//   warp 0      TMA producer: 128x64 tiles of X (and r x 64 tiles of A) into a
 //               3-stage ring (128-byte swizzle, the UMMA K-major layout)
-//   warp 1      owns TMEM (64 columns), issues tcgen05.mma M=128,N=64,K=16 on
-//               each X tile for the LoRA down-projection
+//   warp 1      owns TMEM (r columns, rounded up to a power of two), issues
+//               tcgen05.mma M=128,N=r,K=16 on each X tile for the LoRA
+//               down-projection
 //   warps 2-9   256 row threads: thread = (row, half of each 64-wide tile,
 //               i.e. 32 columns = 8 groups = two 16-bit metadata fields); the
 //               kept values of a tile leave through one TMA store.  (Half rows
@@ -55,16 +56,18 @@ constexpr int kComputeWarps = 8;
 constexpr int kComputeThreads = 32 * kComputeWarps;  // 256
 constexpr int kThreads = 64 + kComputeThreads;        // 320
 constexpr uint32_t kXTileBytes = 128 * 64 * 2;        // 16 KB
-constexpr uint32_t kATileBytes = 64 * 64 * 2;         // 8 KB
 constexpr uint32_t kStoreTileBytes = 128 * 32 * 2;    // 8 KB: 128 rows x 32 kept values
-constexpr uint32_t kTmemCols = 64;
 constexpr uint32_t kBarCompute = 1;                   // named barrier of the row threads
 
-struct __align__(1024) SparsifySmem {
-  uint8_t xring[kStages][kXTileBytes];
-  uint8_t aring[kStages][kATileBytes];
-  uint8_t vstage[2][kStoreTileBytes];  // kept values of one tile, 64-byte swizzle
-  float2 half1[128];                   // partial sums of the second half of each row
+// Shared memory, laid out at run time (the A ring depends on the LoRA rank r):
+//   xring  kStages x 16 KB       X boxes, 128 rows x 64 columns (128-byte swizzle)
+//   aring  kStages x r*128 B     A boxes, r rows x 64 columns (with LoRA only)
+//   vstage 2 x 8 KB              kept values of one box (64-byte swizzle)
+//   ctl    SparsifyCtl           barriers and per-row partials
+// Every tile starts on a 1024-byte boundary (r % 16 == 0 makes r*128 a
+// multiple of 2048).
+struct SparsifyCtl {
+  float2 half1[128];           // partial sums of the second half of each row
   uint64_t full[kStages];
   uint64_t empty[kStages];     // row threads done with a stage (one arrival per warp)
   uint64_t mma_done[kStages];  // the LoRA MMAs done with a stage (tcgen05.commit)
@@ -74,6 +77,28 @@ struct __align__(1024) SparsifySmem {
   uint32_t tmem_base;
   volatile uint32_t abort_flag;
 };
+
+struct SparsifyLayout {
+  uint32_t a_tile;  // bytes of one A box (0 without LoRA)
+  uint32_t aring, vstage, ctl, total;
+};
+
+__host__ __device__ inline SparsifyLayout sparsify_layout(bool lora, int r) {
+  SparsifyLayout l;
+  l.a_tile = lora ? static_cast<uint32_t>(r) * 128u : 0u;
+  l.aring = kStages * kXTileBytes;
+  l.vstage = l.aring + kStages * l.a_tile;
+  l.ctl = l.vstage + 2 * kStoreTileBytes;
+  l.total = l.ctl + static_cast<uint32_t>(sizeof(SparsifyCtl));
+  return l;
+}
+
+// TMEM columns for the LoRA-down accumulator: a power of two >= 32 and >= r
+__host__ __device__ inline uint32_t lora_tmem_cols(int r) {
+  uint32_t c = 32;
+  while (c < static_cast<uint32_t>(r)) c <<= 1;
+  return c;
+}
 
 // acc_lo += |low bf16 of w|, acc_hi += |high bf16 of w|: each half widened to
 // fp32 exactly, the magnitude taken by the add's operand modifier
@@ -124,7 +149,7 @@ __device__ __forceinline__ uint32_t scale_pair(uint32_t w, float s) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
-__device__ __forceinline__ void set_abort(SparsifySmem& sm, uint32_t* status, uint32_t code) {
+__device__ __forceinline__ void set_abort(SparsifyCtl& sm, uint32_t* status, uint32_t code) {
   record_error(status, code);
   sm.abort_flag = 1u;
 }
@@ -132,17 +157,23 @@ __device__ __forceinline__ void set_abort(SparsifySmem& sm, uint32_t* status, ui
 __global__ void __launch_bounds__(kThreads, 2)
 sparsify_kernel(const __grid_constant__ SparsifyLaunch p) {
   extern __shared__ uint8_t smem_raw[];
-  SparsifySmem& sm = *reinterpret_cast<SparsifySmem*>(
+  const bool do_sel = (p.mode & kModeSelect) != 0;
+  const bool do_lora = (p.mode & kModeLora) != 0;
+  const SparsifyLayout lay = sparsify_layout(do_lora, p.r);
+  uint8_t* base = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  SparsifyCtl& sm = *reinterpret_cast<SparsifyCtl*>(base + lay.ctl);
+  uint8_t* const xring = base;
+  uint8_t* const aring = base + lay.aring;
+  uint8_t* const vstage = base + lay.vstage;
 
   const uint32_t warp = warp_id_sync();
   const uint32_t lane = lane_id();
   const uint32_t j = blockIdx.x;  // K range
   const int64_t mb = blockIdx.y;  // row block
   const int nboxes = p.boxes_per_cta;
-  const bool do_sel = (p.mode & kModeSelect) != 0;
-  const bool do_lora = (p.mode & kModeLora) != 0;
   const int64_t kcol0 = static_cast<int64_t>(j) * nboxes * 64;
+  const uint32_t tmem_cols = do_lora ? lora_tmem_cols(p.r) : 0u;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -167,16 +198,16 @@ sparsify_kernel(const __grid_constant__ SparsifyLaunch p) {
     tma_prefetch_desc(&p.tm_x);
     if (do_lora) tma_prefetch_desc(&p.tm_a);
     pdl_wait();
-    const uint32_t tx = kXTileBytes + (do_lora ? kATileBytes : 0u);
+    const uint32_t tx = kXTileBytes + lay.a_tile;
     for (int b = 0; b < preissued; ++b) {
       mbar_arrive_expect_tx(&sm.full[b], tx);
       const int32_t kc = static_cast<int32_t>(kcol0 + 64 * b);
-      tma_load_2d(sm.xring[b], &p.tm_x, &sm.full[b], kc, static_cast<int32_t>(mb * 128));
-      if (do_lora) tma_load_2d(sm.aring[b], &p.tm_a, &sm.full[b], kc, 0);
+      tma_load_2d(xring + b * kXTileBytes, &p.tm_x, &sm.full[b], kc, static_cast<int32_t>(mb * 128));
+      if (do_lora) tma_load_2d(aring + b * lay.a_tile, &p.tm_a, &sm.full[b], kc, 0);
     }
   }
   if (warp == 1 && do_lora) {
-    tmem_alloc(&sm.tmem_base, kTmemCols);
+    tmem_alloc(&sm.tmem_base, tmem_cols);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -189,6 +220,11 @@ sparsify_kernel(const __grid_constant__ SparsifyLaunch p) {
   // the next kernel (finalize_kernel, or the GEMM that combines the partials
   // itself) may begin launching; it waits for this whole grid
   pdl_launch_dependents();
+  // The GEMM of this call claims and publishes each row block through these
+  // words; it reads them only after this grid has completed, and the previous
+  // kernel on the stream (an earlier call's GEMM) has completed before here.
+  if (p.fin_flags != nullptr && blockIdx.x == 0 && blockIdx.y == 0)
+    for (int i = static_cast<int>(threadIdx.x); i < p.fin_nflags; i += kThreads) p.fin_flags[i] = 0u;
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -199,7 +235,7 @@ sparsify_kernel(const __grid_constant__ SparsifyLaunch p) {
     // then (vfree).  The last box's buffer is not needed again.
     if (lane == 0) {
       if (do_sel) tma_prefetch_desc(&p.tm_vals);
-      const uint32_t tx = kXTileBytes + (do_lora ? kATileBytes : 0u);
+      const uint32_t tx = kXTileBytes + lay.a_tile;
       const bool store_rows = mb * 128 < p.M;  // a padding row block has metadata only
       bool ok = !p.stall_test;
       int issued = ok ? preissued : 0;
@@ -215,7 +251,8 @@ sparsify_kernel(const __grid_constant__ SparsifyLaunch p) {
               break;
             }
             if (store_rows) {
-              tma_store_2d(&p.tm_vals, sm.vstage[prev & 1], static_cast<int32_t>((kcol0 + 64 * prev) / 2),
+              tma_store_2d(&p.tm_vals, vstage + (prev & 1) * kStoreTileBytes,
+                           static_cast<int32_t>((kcol0 + 64 * prev) / 2),
                            static_cast<int32_t>(mb * 128));
               bulk_commit();
               // the store of box prev - 1 has read its buffer (this one may still
@@ -238,8 +275,9 @@ sparsify_kernel(const __grid_constant__ SparsifyLaunch p) {
         if (b >= preissued && b < nboxes) {
           mbar_arrive_expect_tx(&sm.full[slot], tx);
           const int32_t kc = static_cast<int32_t>(kcol0 + 64 * b);
-          tma_load_2d(sm.xring[slot], &p.tm_x, &sm.full[slot], kc, static_cast<int32_t>(mb * 128));
-          if (do_lora) tma_load_2d(sm.aring[slot], &p.tm_a, &sm.full[slot], kc, 0);
+          tma_load_2d(xring + slot * kXTileBytes, &p.tm_x, &sm.full[slot], kc,
+                      static_cast<int32_t>(mb * 128));
+          if (do_lora) tma_load_2d(aring + slot * lay.a_tile, &p.tm_a, &sm.full[slot], kc, 0);
           ++issued;
         }
       }
@@ -254,7 +292,7 @@ sparsify_kernel(const __grid_constant__ SparsifyLaunch p) {
   } else if (warp == 1) {
     // ------------------------------------------------------------ LoRA-down MMA
     if (do_lora && lane == 0) {
-      const uint32_t idesc = make_idesc_bf16(128, kLoraRank, false);
+      const uint32_t idesc = make_idesc_bf16(128, static_cast<uint32_t>(p.r), false);
       const uint32_t t_tmem = sm.tmem_base;
       for (int b = 0; b < nboxes; ++b) {
         const int slot = b % kStages;
@@ -265,8 +303,8 @@ sparsify_kernel(const __grid_constant__ SparsifyLaunch p) {
           break;
         }
         tc_fence_after();
-        const uint32_t xa = smem_u32(sm.xring[slot]);
-        const uint32_t aa = smem_u32(sm.aring[slot]);
+        const uint32_t xa = smem_u32(xring + slot * kXTileBytes);
+        const uint32_t aa = smem_u32(aring + slot * lay.a_tile);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
           const uint64_t da = make_sdesc(xa + 32 * kk, 16, 1024, kSw128);
@@ -321,7 +359,7 @@ sparsify_kernel(const __grid_constant__ SparsifyLaunch p) {
         ok = false;
       }
       if (!__all_sync(0xffffffffu, ok)) break;
-      const uint8_t* tile = sm.xring[slot];
+      const uint8_t* tile = xring + slot * kXTileBytes;
       const uint4 v0 = *reinterpret_cast<const uint4*>(tile + ld_off0);
       const uint4 v1 = *reinterpret_cast<const uint4*>(tile + ld_off1);
       const uint4 v2 = *reinterpret_cast<const uint4*>(tile + ld_off2);
@@ -347,8 +385,9 @@ sparsify_kernel(const __grid_constant__ SparsifyLaunch p) {
         ok = false;
       }
       if (!__all_sync(0xffffffffu, ok)) break;
-      *reinterpret_cast<uint4*>(sm.vstage[b & 1] + vst_off0) = make_uint4(kw[0], kw[1], kw[2], kw[3]);
-      *reinterpret_cast<uint4*>(sm.vstage[b & 1] + vst_off1) = make_uint4(kw[4], kw[5], kw[6], kw[7]);
+      uint8_t* const vbuf = vstage + (b & 1) * kStoreTileBytes;
+      *reinterpret_cast<uint4*>(vbuf + vst_off0) = make_uint4(kw[0], kw[1], kw[2], kw[3]);
+      *reinterpret_cast<uint4*>(vbuf + vst_off1) = make_uint4(kw[4], kw[5], kw[6], kw[7]);
       fence_proxy_async_smem();
       // release the stage only after everything derived from it has been
       // produced: an arrive does not wait for this warp's loads in flight
@@ -375,17 +414,16 @@ sparsify_kernel(const __grid_constant__ SparsifyLaunch p) {
     const int64_t grow = mb * 128 + row;
     if (!sm.abort_flag && mbar_wait(&sm.tdone, 0)) {
       tc_fence_after();
-      float4* dst = reinterpret_cast<float4*>(p.tpart + (static_cast<size_t>(j) * p.M + grow) * kLoraRank);
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        uint32_t r[32];
-        tmem_ld_32x32b_x32(sm.tmem_base + ((32u * (warp & 3)) << 16) + 32u * h, r);
+      float4* dst = reinterpret_cast<float4*>(p.tpart + (static_cast<size_t>(j) * p.M + grow) * p.r);
+      for (int c = 0; c < p.r; c += 16) {
+        uint32_t r[16];
+        tmem_ld_32x32b_x16(sm.tmem_base + ((32u * (warp & 3)) << 16) + static_cast<uint32_t>(c), r);
         tmem_ld_wait();
         if (grow < p.M) {
 #pragma unroll
-          for (int c = 0; c < 32; c += 4)
-            dst[(32 * h + c) / 4] = make_float4(__uint_as_float(r[c]), __uint_as_float(r[c + 1]),
-                                                __uint_as_float(r[c + 2]), __uint_as_float(r[c + 3]));
+          for (int e = 0; e < 16; e += 4)
+            dst[(c + e) / 4] = make_float4(__uint_as_float(r[e]), __uint_as_float(r[e + 1]),
+                                           __uint_as_float(r[e + 2]), __uint_as_float(r[e + 3]));
         }
       }
       tc_fence_before();
@@ -395,14 +433,14 @@ sparsify_kernel(const __grid_constant__ SparsifyLaunch p) {
   }
 
   __syncthreads();
-  if (warp == 1 && do_lora) tmem_dealloc(sm.tmem_base, kTmemCols);
+  if (warp == 1 && do_lora) tmem_dealloc(sm.tmem_base, tmem_cols);
 }
 
 // One warp per row: s from the C partial sums, T from the C partial products
-// (fixed order), T written as bf16(T / s) when `divide`.
+// (fixed order), T [M, r] written as bf16(T / s) when `divide`.
 __global__ void __launch_bounds__(256)
 finalize_kernel(const float2* __restrict__ lpart, const float* __restrict__ tpart, int64_t M,
-                int C, int do_scale, int do_lora, int divide, float* __restrict__ row_scale,
+                int C, int r, int do_scale, int do_lora, int divide, float* __restrict__ row_scale,
                 __nv_bfloat16* __restrict__ t_out) {
   pdl_launch_dependents();
   pdl_wait();  // the partials of sparsify_kernel
@@ -429,25 +467,27 @@ finalize_kernel(const float2* __restrict__ lpart, const float* __restrict__ tpar
     if (lane == 0) row_scale[row] = s;
   }
   if (do_lora) {
-    float2 v[kMaxSplit];  // columns 2*lane, 2*lane+1 of each partial
+    // columns 2c, 2c + 1 of each partial, c = lane, lane + 32, ...
+    for (int c = static_cast<int>(lane); 2 * c < r; c += 32) {
+      float2 v[kMaxSplit];
 #pragma unroll
-    for (int j = 0; j < kMaxSplit; ++j)
-      if (j < C)
-        v[j] = __ldcg(reinterpret_cast<const float2*>(
-                          tpart + (static_cast<size_t>(j) * M + row) * kLoraRank) + lane);
-    float a0 = 0.f, a1 = 0.f;
+      for (int j = 0; j < kMaxSplit; ++j)
+        if (j < C)
+          v[j] = __ldcg(reinterpret_cast<const float2*>(tpart + (static_cast<size_t>(j) * M + row) * r) + c);
+      float a0 = 0.f, a1 = 0.f;
 #pragma unroll
-    for (int j = 0; j < kMaxSplit; ++j) {
-      if (j < C) {
-        a0 = __fadd_rn(a0, v[j].x);
-        a1 = __fadd_rn(a1, v[j].y);
+      for (int j = 0; j < kMaxSplit; ++j) {
+        if (j < C) {
+          a0 = __fadd_rn(a0, v[j].x);
+          a1 = __fadd_rn(a1, v[j].y);
+        }
       }
+      if (divide) {
+        a0 = __fdiv_rn(a0, s);
+        a1 = __fdiv_rn(a1, s);
+      }
+      reinterpret_cast<__nv_bfloat162*>(t_out + row * r)[c] = __floats2bfloat162_rn(a0, a1);
     }
-    if (divide) {
-      a0 = __fdiv_rn(a0, s);
-      a1 = __fdiv_rn(a1, s);
-    }
-    reinterpret_cast<__nv_bfloat162*>(t_out + row * kLoraRank)[lane] = __floats2bfloat162_rn(a0, a1);
   }
 }
 
@@ -469,7 +509,9 @@ rescale_kernel(uint4* __restrict__ vals, const float* __restrict__ row_scale, in
 
 }  // namespace
 
-size_t sparsify_smem_bytes() { return sizeof(SparsifySmem) + 1024; }
+size_t sparsify_smem_bytes(int mode, int r) {
+  return sparsify_layout((mode & kModeLora) != 0, r).total + 1024;  // + alignment slack
+}
 
 // K ranges per row block: the largest C <= kMaxSplit dividing the 64-column
 // boxes of a row such that C * ceil(M/128) CTAs fit in one wave (2 per SM).
@@ -486,20 +528,19 @@ int choose_sparsify_split(int64_t M, int64_t K, int num_sms) {
 }
 
 cudaError_t launch_sparsify(const SparsifyLaunch& p, cudaStream_t stream) {
-  const size_t smem = sparsify_smem_bytes();
-  static int configured_device = -1;
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (configured_device != dev) {
-    cudaError_t e = cudaFuncSetAttribute(sparsify_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem));
-    if (e != cudaSuccess) return e;
-    configured_device = dev;
-  }
+  const size_t smem = sparsify_smem_bytes(p.mode, p.r);
+  // the largest layout (r = kLoraRankMax) is allowed once per device
+  static std::once_flag once[64];
+  static cudaError_t configured[64];
+  cudaError_t e = once_per_device(once, configured, []() {
+    return cudaFuncSetAttribute(sparsify_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                static_cast<int>(sparsify_smem_bytes(kModeSelect | kModeLora, kLoraRankMax)));
+  });
+  if (e != cudaSuccess) return e;
   // metadata row blocks come in pairs: the block past M (if any) gets the
   // pattern of all-zero rows, so a CTA pair of the GEMM never reads garbage
   const dim3 grid(static_cast<unsigned>(p.split), static_cast<unsigned>(meta_row_blocks(p.M)), 1);
-  cudaError_t e = launch_after_previous(sparsify_kernel, grid, dim3(kThreads), smem, stream, p);
+  e = launch_after_previous(sparsify_kernel, grid, dim3(kThreads), smem, stream, p);
   if (e != cudaSuccess || p.skip_finalize) return e;
   const bool do_sel = (p.mode & kModeSelect) != 0;
   const bool do_lora = (p.mode & kModeLora) != 0;
@@ -507,7 +548,7 @@ cudaError_t launch_sparsify(const SparsifyLaunch& p, cudaStream_t stream) {
   const unsigned fin_blocks = static_cast<unsigned>((p.M + 7) / 8);
   e = launch_after_previous(finalize_kernel, dim3(fin_blocks), dim3(256), 0, stream,
                             static_cast<const float2*>(p.lpart), static_cast<const float*>(p.tpart),
-                            p.M, p.split, do_sel ? 1 : 0, do_lora ? 1 : 0,
+                            p.M, p.split, p.r, do_sel ? 1 : 0, do_lora ? 1 : 0,
                             (do_sel && !scaled) ? 1 : 0, p.row_scale,
                             static_cast<__nv_bfloat16*>(p.t_out));
   if (e != cudaSuccess || !(do_sel && scaled)) return e;

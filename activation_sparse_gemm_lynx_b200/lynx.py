@@ -51,6 +51,7 @@ def library():
             "lynx_status_string": ([i32], ctypes.c_char_p),
             "lynx_version": ([], i32),
             "lynx_lora_rank": ([], i32),
+            "lynx_lora_rank_supported": ([i64], i32),
             "lynx_vals_bytes": ([i64, i64], sz),
             "lynx_meta_bytes": ([i64, i64], sz),
             "lynx_workspace_bytes": ([i64, i64, i64, i64], sz),
@@ -70,6 +71,7 @@ def library():
             "lynx_meta_canonical_to_hw": ([p, p, i64, i64], i32),
             "lynx_debug_set_stall": ([i32], i32),
             "lynx_profile_set_split_event": ([p], p),
+            "lynx_profile_set_part": ([i32], i32),
         }
         for name, (args, res) in sigs.items():
             f = getattr(lib, name)
@@ -95,7 +97,13 @@ def lynx_version():
 
 
 def lynx_lora_rank():
+    """The LoRA rank the RT-Lynx pages use (64), the default of these bindings."""
     return library().lynx_lora_rank()
+
+
+def lynx_lora_rank_supported(r):
+    """True if the kernels accept LoRA rank r (r % 16 == 0, 16 <= r <= 256)."""
+    return bool(library().lynx_lora_rank_supported(int(r)))
 
 
 def lynx_vals_bytes(M, K):
@@ -406,6 +414,13 @@ def lynx_profile_set_split_event(event):
     every later lynx_linear call (see include/lynx.h)."""
     handle = None if event is None else ctypes.c_void_p(event.cuda_event)
     return library().lynx_profile_set_split_event(handle)
+
+
+def lynx_profile_set_part(part):
+    """Profiling hook: 1 = only the sparsify / LoRA-down pass of each later
+    lynx_linear call, 2 = only what follows it, 0 = the whole layer (see
+    include/lynx.h).  Returns the previous part."""
+    return library().lynx_profile_set_part(int(part))
 
 
 def lynx_debug_set_stall(enable):

@@ -36,10 +36,12 @@ sys.path.insert(0, ROOT)
 METRIC = "sparse-act linear dense-equiv TFLOP/s (2MNK/t) & speedup vs dense bf16 GEMM"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
-# DRAM bytes (read + write) per launch of the sparse GEMM kernel, from one ncu
-# capture of the kernel as it stands (dram__bytes_read.sum + dram__bytes_write.sum);
-# a workload that has not been captured reports null.
-GEMM_DRAM_TRAFFIC = {"mlp_up": 103.04e6 + 83.54e6}
+# DRAM bytes (read + write) per launch of the sparse GEMM kernel from one ncu
+# capture (dram__bytes_read.sum + dram__bytes_write.sum), with the hash of the
+# GEMM's sources at the capture: the bench reports the figure only while the
+# sources still hash the same, else null ("stale").
+GEMM_SOURCES = ("gemm_pair_kernel.cu", "lynx_ptx.cuh", "lynx_internal.h", "lynx_act.cuh")
+GEMM_DRAM_TRAFFIC = {}
 
 def uses_pair_gemm(M, N, K):
     """The library's choice: the CTA-pair GEMM unless the shape cannot feed it."""
@@ -75,6 +77,8 @@ def parse_args(argv=None):
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="approximate CPU time of the oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-per-config", action="store_true",
+                    help="skip the per_config block (the other DiT shapes)")
     ap.add_argument("--only-linear", action="store_true",
                     help="time the layer only (no comparisons, e2e or CPU baseline); "
                          "the short launch sequence used for ncu captures")
@@ -309,11 +313,139 @@ def run_reference(args):
     return 0
 
 
+class LayerTimer:
+    """Device-resident inputs of one workload and the timing loops over them
+    (CUDA events on the launching stream, L2 flushed before every step)."""
+
+    def __init__(self, name, rank, act_name, flush):
+        import numpy as np
+        import torch
+
+        from activation_sparse_gemm_lynx_b200 import lynx, workloads
+
+        self.lynx, self.torch = lynx, torch
+        self.shape = workloads.CONFIGS[name]
+        M, N, K, r = self.shape.M, self.shape.N, self.shape.K, self.shape.r
+        self.inp = workloads.make_rank_inputs(name, rank)
+
+        def dev(a):
+            return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).cuda()
+
+        self.X, self.W, self.bias, self.A, self.B = (dev(self.inp[k]) for k in ("X", "W", "bias", "A", "B"))
+        self.Y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+        self.Yd = torch.empty_like(self.Y)
+        self.ws = torch.empty(lynx.lynx_workspace_bytes(M, N, K, r), dtype=torch.uint8, device="cuda")
+        self.flush = flush
+        self.act = {"none": lynx.LYNX_ACT_NONE, "gelu_tanh": lynx.LYNX_ACT_GELU_TANH}[act_name]
+
+    def step_linear(self, skip=False):
+        if self.act == self.lynx.LYNX_ACT_NONE and not skip:
+            self.lynx.lynx_linear(self.X, self.W, self.bias, self.A, self.B, Y=self.Y, workspace=self.ws)
+        else:
+            self.lynx.lynx_linear_act(self.X, self.W, self.bias, self.A, self.B, skip_sparsify=skip,
+                                      act=self.act, Y=self.Y, workspace=self.ws)
+
+    def step_dense_torch(self):
+        self.torch.matmul(self.X, self.W.t(), out=self.Yd)
+        if self.act != self.lynx.LYNX_ACT_NONE:
+            self.torch.nn.functional.gelu(self.Yd, approximate="tanh")
+
+    def step_unfused_act(self):
+        # the plain layer, then the activation as a pass of its own over Y
+        self.lynx.lynx_linear(self.X, self.W, self.bias, self.A, self.B, Y=self.Y, workspace=self.ws)
+        self.torch.nn.functional.gelu(self.Y, approximate="tanh")
+
+    def timed(self, step, n, split=False, part=0):
+        """Per-step device times (ms) of n steps, L2 flushed before each.  With
+        split, also the times up to and after the library's split event; with
+        part 1 / 2, lynx_linear runs only its first kernel / the rest."""
+        torch, lynx = self.torch, self.lynx
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(n)]
+        for trio in ev:        # create the CUDA events up front
+            for e in trio:
+                e.record()
+        torch.cuda.synchronize()
+        lynx.lynx_profile_set_part(part)
+        try:
+            for i in range(n):
+                self.flush.zero_()
+                if split:
+                    lynx.lynx_profile_set_split_event(ev[i][1])
+                ev[i][0].record()
+                step()
+                ev[i][2].record()
+        finally:
+            lynx.lynx_profile_set_split_event(None)
+            lynx.lynx_profile_set_part(0)
+        torch.cuda.synchronize()
+        tot = [ev[i][0].elapsed_time(ev[i][2]) for i in range(n)]
+        if split:
+            first = [ev[i][0].elapsed_time(ev[i][1]) for i in range(n)]
+            second = [ev[i][1].elapsed_time(ev[i][2]) for i in range(n)]
+            return tot, first, second
+        return tot
+
+    def parts(self, n):
+        """Time of the layer's parts, each run alone (means over n steps):
+        the sparsify / LoRA-down kernel (events around that one launch), the
+        GEMM (from an event recorded after the reset of its state words to the
+        end), and the two kernels of a call split by an event between them."""
+        mean = statistics.mean
+        sp_alone = mean(self.timed(self.step_linear, n, part=1))
+        _, _, gemm_alone = self.timed(self.step_linear, n, split=True, part=2)
+        split_tot, split_sp, split_gemm = self.timed(self.step_linear, n, split=True)
+        return {"sparsify_kernel": sp_alone, "gemm_kernel": mean(gemm_alone),
+                "linear_split": mean(split_tot), "split_first": mean(split_sp),
+                "split_second": mean(split_gemm)}
+
+
+def src_hash(files):
+    """Short hash of the named CUDA sources (the build a stored ncu figure belongs to)."""
+    import hashlib
+
+    h = hashlib.sha256()
+    for f in files:
+        with open(os.path.join(ROOT, "activation_sparse_gemm_lynx_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:12]
+
+
+def stored_gemm_traffic(workload):
+    """ncu's DRAM bytes per launch of the GEMM for this workload, if the stored
+    capture was taken on the GEMM sources as they stand; else (None, why)."""
+    rec = GEMM_DRAM_TRAFFIC.get(workload)
+    if rec is None:
+        return None, "not captured for this workload"
+    now = src_hash(GEMM_SOURCES)
+    if rec["src"] != now:
+        return None, f"stale: captured on sources {rec['src']}, kernel now {now}"
+    return rec["bytes"], f"ncu capture of {rec['captured']} (sources {rec['src']})"
+
+
+def layer_summary(lt, ms_linear, parts, dense_ms, peaks, clock_info=None):
+    M, N, K, r = lt.shape.M, lt.shape.N, lt.shape.K, lt.shape.r
+    flops = 2.0 * M * N * K
+    sparse_peak = 2.0 * peaks["bf16_tflops"]
+    gemm_tflops = flops / (parts["gemm_kernel"] * 1e-3) / 1e12
+    out = {
+        "value": flops / (ms_linear * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": ms_linear,
+        "M": M, "N": N, "K": K, "r": r,
+        "speedup_vs_dense_bf16": dense_ms / ms_linear,
+        "sparsify_overhead": max(0.0, 1.0 - parts["gemm_kernel"] / ms_linear),
+        "gemm_frac": gemm_tflops / sparse_peak,
+        "gemm_tflops": gemm_tflops,
+        "ms": {"sparsify_kernel": parts["sparsify_kernel"], "gemm_kernel": parts["gemm_kernel"],
+               "dense_torch_matmul": dense_ms},
+    }
+    if clock_info is not None:
+        out["clocks"] = clock_info
+    return out
+
+
 def run_lynx(args):
-    import numpy as np
     import torch
 
-    from activation_sparse_gemm_lynx_b200 import lynx, workloads
+    from activation_sparse_gemm_lynx_b200 import lynx
 
     rank, local_rank, world = dist_env()
     if world != args.gpus:
@@ -325,42 +457,13 @@ def run_lynx(args):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local_rank))
     lynx.library()
-
-    shape = workloads.CONFIGS[args.workload]
-    M, N, K, r = shape.M, shape.N, shape.K, shape.r
-    inp = workloads.make_rank_inputs(args.workload, rank)
-
-    def dev(a):
-        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).cuda()
-
-    X, W, bias, A, B = (dev(inp[k]) for k in ("X", "W", "bias", "A", "B"))
-    Y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
-    Yd = torch.empty_like(Y)
-    ws = torch.empty(lynx.lynx_workspace_bytes(M, N, K, r), dtype=torch.uint8, device="cuda")
     flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.int32, device="cuda")
-    Xh = torch.from_numpy(inp["X"].view(np.int16)).view(torch.bfloat16).pin_memory()
+    lt = LayerTimer(args.workload, rank, args.act, flush)
+    shape = lt.shape
+    M, N, K, r = shape.M, shape.N, shape.K, shape.r
+    Xh = torch.from_numpy(lt.inp["X"].view("int16")).view(torch.bfloat16).pin_memory()
     Yh = torch.empty((M, N), dtype=torch.bfloat16).pin_memory()
-
-    act = {"none": lynx.LYNX_ACT_NONE, "gelu_tanh": lynx.LYNX_ACT_GELU_TANH}[args.act]
-
-    def step_linear():
-        if act == lynx.LYNX_ACT_NONE:
-            lynx.lynx_linear(X, W, bias, A, B, Y=Y, workspace=ws)
-        else:
-            lynx.lynx_linear_act(X, W, bias, A, B, act=act, Y=Y, workspace=ws)
-
-    def step_dense_lynx():
-        lynx.lynx_linear_act(X, W, bias, A, B, skip_sparsify=True, act=act, Y=Y, workspace=ws)
-
-    def step_dense_torch():
-        torch.matmul(X, W.t(), out=Yd)
-        if act != lynx.LYNX_ACT_NONE:
-            torch.nn.functional.gelu(Yd, approximate="tanh")
-
-    def step_unfused_act():
-        # the plain layer, then the activation as a pass of its own over Y
-        lynx.lynx_linear(X, W, bias, A, B, Y=Y, workspace=ws)
-        torch.nn.functional.gelu(Y, approximate="tanh")
+    act = lt.act
 
     ws_host = torch.empty(lynx.lynx_linear_host_workspace_bytes(M, N, K, r), dtype=torch.uint8,
                           device="cuda")
@@ -369,56 +472,30 @@ def run_lynx(args):
         # the C-ABI call on host buffers: copies in, the layer and copies out,
         # pipelined over row chunks inside the library
         if act == lynx.LYNX_ACT_NONE:
-            lynx.lynx_linear_host(Xh, W, bias, A, B, Y_host=Yh, workspace=ws_host)
+            lynx.lynx_linear_host(Xh, lt.W, lt.bias, lt.A, lt.B, Y_host=Yh, workspace=ws_host)
         else:
-            lynx.lynx_linear_host_act(Xh, W, bias, A, B, act=act, Y_host=Yh, workspace=ws_host)
-
-    def timed(step, n, split=False):
-        """Per-step device times (ms) of n steps, L2 flushed before each."""
-        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(n)]
-        for trio in ev:        # create the CUDA events up front
-            for e in trio:
-                e.record()
-        torch.cuda.synchronize()
-        for i in range(n):
-            flush.zero_()
-            if split:
-                lynx.lynx_profile_set_split_event(ev[i][1])
-            ev[i][0].record()
-            step()
-            ev[i][2].record()
-        if split:
-            lynx.lynx_profile_set_split_event(None)
-        torch.cuda.synchronize()
-        tot = [ev[i][0].elapsed_time(ev[i][2]) for i in range(n)]
-        if split:
-            first = [ev[i][0].elapsed_time(ev[i][1]) for i in range(n)]
-            second = [ev[i][1].elapsed_time(ev[i][2]) for i in range(n)]
-            return tot, first, second
-        return tot
+            lynx.lynx_linear_host_act(Xh, lt.W, lt.bias, lt.A, lt.B, act=act, Y_host=Yh,
+                                      workspace=ws_host)
 
     # warm-up (untimed)
     for _ in range(args.warmup):
-        step_linear()
+        lt.step_linear()
     torch.cuda.synchronize()
     st, code = lynx.lynx_check_error()
     if st != lynx.LYNX_OK:
         raise RuntimeError(f"device status after warm-up: {st} code {code:#x}")
 
-    # breakdown in a loop of its own, before the timed steps: an event recorded
-    # between the sparsify pass and the GEMM keeps the GEMM's launch from
-    # overlapping the pass's tail, so the headline loop runs without it
+    # the parts of the layer, each in a loop of its own before the timed steps
+    # (an event between the kernels keeps the GEMM's launch from overlapping the
+    # pass's tail, so the headline loop runs without it)
     ncmp = max(3, min(args.steps, 50))
-    split_tot, t_sp, t_gemm = timed(step_linear, ncmp, split=True)
-    split_ms = statistics.mean(split_tot)
-    sp_ms = statistics.mean(t_sp)
-    gemm_ms = statistics.mean(t_gemm)
+    parts = lt.parts(ncmp)
 
     clocks = ClockSampler(local_rank)
     barrier(world)
     torch.cuda.synchronize()
     clocks.start()
-    tot = timed(step_linear, args.steps)
+    tot = lt.timed(lt.step_linear, args.steps)
     torch.cuda.synchronize()
     clock_info = clocks.stop()
     barrier(world)
@@ -434,34 +511,38 @@ def run_lynx(args):
 
             dist.destroy_process_group()
         if rank == 0:
-            print(json.dumps({"metric": METRIC, "ms_per_step": ms_step, "sparsify_ms": sp_ms,
-                              "gemm_ms": gemm_ms, "n_gpus": world, "steps": args.steps,
-                              "warmup": args.warmup, "only_linear": True}), flush=True)
+            print(json.dumps({"metric": METRIC, "ms_per_step": ms_step,
+                              "sparsify_ms": parts["sparsify_kernel"], "gemm_ms": parts["gemm_kernel"],
+                              "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+                              "only_linear": True}), flush=True)
         return 0
 
     # comparisons (same process, same loop structure)
     for _ in range(3):
-        step_dense_torch()
-    dense_ms = max_over_ranks(statistics.mean(timed(step_dense_torch, ncmp)), world)
+        lt.step_dense_torch()
+    dense_ms = max_over_ranks(statistics.mean(lt.timed(lt.step_dense_torch, ncmp)), world)
     for _ in range(3):
-        step_dense_lynx()
-    lynx_dense_ms = max_over_ranks(statistics.mean(timed(step_dense_lynx, ncmp)), world)
+        lt.step_linear(skip=True)
+    lynx_dense_ms = max_over_ranks(statistics.mean(lt.timed(lambda: lt.step_linear(skip=True), ncmp)),
+                                   world)
     for _ in range(3):
         step_e2e()
-    e2e_ms = max_over_ranks(statistics.mean(timed(step_e2e, ncmp)), world)
+    e2e_ms = max_over_ranks(statistics.mean(lt.timed(step_e2e, ncmp)), world)
     unfused_ms = None
     if act != lynx.LYNX_ACT_NONE:
         for _ in range(3):
-            step_unfused_act()
-        unfused_ms = max_over_ranks(statistics.mean(timed(step_unfused_act, ncmp)), world)
+            lt.step_unfused_act()
+        unfused_ms = max_over_ranks(statistics.mean(lt.timed(lt.step_unfused_act, ncmp)), world)
+    parts = {k: max_over_ranks(v, world) for k, v in parts.items()}
 
     flops = 2.0 * M * N * K
     peaks = load_peaks()
     sparse_peak = 2.0 * peaks["bf16_tflops"]
-    gemm_tflops = flops / (gemm_ms * 1e-3) / 1e12
+    gemm_tflops = flops / (parts["gemm_kernel"] * 1e-3) / 1e12
     sp_bytes = 2 * M * K + M * K + lynx.lynx_meta_bytes(M, K) + 2 * M * r + 4 * M + 2 * r * K
-    sp_gbs = sp_bytes / (sp_ms * 1e-3) / 1e9
-    traffic = GEMM_DRAM_TRAFFIC.get(args.workload)
+    sp_gbs = sp_bytes / (parts["sparsify_kernel"] * 1e-3) / 1e9
+    traffic, traffic_note = stored_gemm_traffic(args.workload) if act == lynx.LYNX_ACT_NONE \
+        else (None, "not captured with the epilogue activation")
 
     result = {
         "metric": METRIC,
@@ -484,23 +565,26 @@ def run_lynx(args):
             "parallelism": f"dp{world} (independent token-row batches per GPU, no collective)",
         },
         "speedup_vs_dense_bf16": dense_ms / ms_step,
-        "sparsify_overhead": sp_ms / split_ms,
-        "breakdown_ms": {"linear": ms_step, "linear_split": split_ms, "sparsify_pass": sp_ms,
-                         "sparse_gemm": gemm_ms,
+        "sparsify_overhead": max(0.0, 1.0 - parts["gemm_kernel"] / ms_step),
+        "overhead_note": "1 - t(GEMM kernel alone) / t(layer): the time the layer adds to its GEMM",
+        "breakdown_ms": {"linear": ms_step, "sparsify_kernel": parts["sparsify_kernel"],
+                         "gemm_kernel": parts["gemm_kernel"], "linear_split": parts["linear_split"],
+                         "split_sparsify_pass": parts["split_first"], "split_gemm": parts["split_second"],
                          "dense_torch_matmul": dense_ms, "lynx_dense_path": lynx_dense_ms},
         "roofline": {
             "bound": "tensor", "kernel": gemm_kernel_name(M, N, K),
             "achieved": gemm_tflops, "peak": sparse_peak, "unit": "TFLOP/s",
-            "frac": gemm_tflops / sparse_peak, "traffic": traffic,
+            "frac": gemm_tflops / sparse_peak, "traffic": traffic, "traffic_note": traffic_note,
             "peak_note": f"2 x {peaks['source']} dense bf16 burst ({peaks['bf16_tflops']} TFLOP/s); "
                          "2:4 sparse runs at twice the dense rate",
-            "work": "2*M*N*K dense-equivalent flops per launch",
+            "work": "2*M*N*K dense-equivalent flops per launch; time: the GEMM launched alone",
         },
         "roofline_sparsify": {
             "bound": "hbm", "kernel": "sparsify_kernel", "achieved": sp_gbs,
             "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": sp_gbs / peaks["hbm_gbs"],
             "traffic": None,
-            "work": "X read 2MK + vals MK + meta MK/8 + T 2Mr + s 4M + A 2rK bytes",
+            "work": "algorithmic bytes X read 2MK + vals MK + meta MK/8 + T 2Mr + s 4M + A 2rK; "
+                    "time: the kernel launched alone",
         },
         "e2e": {"value": aggregate_tflops(flops, e2e_ms, world), "unit": "TFLOP/s",
                 "h2d_bytes_per_step": 2 * M * K, "d2h_bytes_per_step": 2 * M * N,
@@ -515,11 +599,40 @@ def run_lynx(args):
         result["config"]["act"] = args.act
         result["speedup_vs_unfused_act"] = unfused_ms / ms_step
         result["breakdown_ms"]["linear_then_separate_act"] = unfused_ms
-        result["breakdown_ms"]["dense_torch_matmul"] = dense_ms
         result["dense_note"] = "torch.matmul then torch GELU (tanh) as a separate pass"
 
+    # the other DiT shapes of the same targets, measured in this run the same
+    # way (fewer steps); the headline stays the selected workload
+    if not args.no_per_config and act == lynx.LYNX_ACT_NONE:
+        per = {}
+        for name in ("attn_out", "mlp_up", "mlp_down"):
+            if name == args.workload:
+                per[name] = layer_summary(lt, ms_step, parts, dense_ms, peaks, clock_info)
+                continue
+            other = LayerTimer(name, rank, "none", flush)
+            for _ in range(max(3, args.warmup)):
+                other.step_linear()
+            torch.cuda.synchronize()
+            o_parts = {k: max_over_ranks(v, world) for k, v in other.parts(ncmp).items()}
+            ck = ClockSampler(local_rank)
+            barrier(world)
+            torch.cuda.synchronize()
+            ck.start()
+            o_ms = max_over_ranks(statistics.mean(other.timed(other.step_linear, ncmp)), world)
+            o_clock = ck.stop()
+            for _ in range(3):
+                other.step_dense_torch()
+            o_dense = max_over_ranks(statistics.mean(other.timed(other.step_dense_torch, ncmp)), world)
+            per[name] = layer_summary(other, o_ms, o_parts, o_dense, peaks, o_clock)
+            per[name]["steps"] = ncmp
+            del other
+        st, code = lynx.lynx_check_error()
+        if st != lynx.LYNX_OK:
+            raise RuntimeError(f"device status after the per-config runs: {st} code {code:#x}")
+        result["per_config"] = per
+
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        result["cpu_baseline"] = cpu_baseline(inp, shape, args.cpu_seconds, act=args.act)
+        result["cpu_baseline"] = cpu_baseline(lt.inp, shape, args.cpu_seconds, act=args.act)
 
     if world > 1:
         import torch.distributed as dist

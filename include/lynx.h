@@ -13,8 +13,9 @@
  *     Top-K).  The kept values are multiplied by the norm-compensation factor
  *     s = sum|x| / sum|kept| of the row, computed in fp32 (section 03.1; ai-feeds
  *     summary, core module 1), and rounded to bf16.
- *   - (X A^T) B^T: LoRA residual of rank r = 64 on the dense X, frozen W
- *     (section 03.2; neuraltrendhub summary: rank 64).
+ *   - (X A^T) B^T: LoRA residual of rank r on the dense X, frozen W (section
+ *     03.2; the neuraltrendhub summary gives rank 64, the pages' setting).  Any
+ *     r with r % 16 == 0 and 16 <= r <= 256 is accepted.
  *   - skip_sparsify: the layer stays dense, S(X) = X (section 03.3, selective
  *     layer skipping).
  *   - The sparse product runs on sparse tensor cores (tcgen05.mma.sp) with the
@@ -31,11 +32,14 @@
  *   - Return value: a lynx_status.  Host-side checks run before anything is
  *     enqueued: on failure nothing is launched and no buffer is touched.
  *     Device-side failures (a bounded wait that gave up) are recorded in a
- *     per-device status word that lynx_check_error reports.
+ *     status word of the stream the call was enqueued on, which
+ *     lynx_check_error(stream) reports; a CUDA graph captured from a stream
+ *     keeps recording into that stream's word when it is replayed.
  *   - Inputs must be finite; NaN/Inf inputs give unspecified (but memory-safe)
  *     results.
  *   - Shapes: M >= 1 tokens, K >= 64 with K % 64 == 0, N >= 8 with N % 8 == 0,
- *     r = 64 when a LoRA branch is given.  Every pointer 16-byte aligned.
+ *     and, when a LoRA branch is given, 16 <= r <= 256 with r % 16 == 0.
+ *     Every pointer 16-byte aligned.
  *   - Thread safety: calls from several host threads on different streams are
  *     safe.  Calls whose device work overlaps must not share output buffers or
  *     a workspace.
@@ -59,7 +63,7 @@ extern "C" {
 typedef enum lynx_status {
   LYNX_OK = 0,
   LYNX_ERR_INVALID_ARG = 1,         /* null pointer, A without B, bad flag */
-  LYNX_ERR_UNSUPPORTED_SHAPE = 2,   /* M < 1, K % 64, N % 8, r != 64, ... */
+  LYNX_ERR_UNSUPPORTED_SHAPE = 2,   /* M < 1, K % 64, N % 8, r % 16, r > 256, ... */
   LYNX_ERR_MISALIGNED = 3,          /* a pointer not 16-byte aligned */
   LYNX_ERR_WORKSPACE_TOO_SMALL = 4, /* workspace_bytes < lynx_workspace_bytes() */
   LYNX_ERR_CUDA = 5,                /* a CUDA runtime/driver call failed */
@@ -72,8 +76,14 @@ LYNX_API const char* lynx_status_string(int status);
 /* ABI version: (major << 16) | minor. */
 LYNX_API int lynx_version(void);
 
-/* Rank of the LoRA branch the kernels implement (64). */
+/* The LoRA rank the RT-Lynx pages use (64); the bindings' default. */
 LYNX_API int lynx_lora_rank(void);
+
+/* 1 if the kernels accept LoRA rank r (r % 16 == 0 and 16 <= r <= 256), else 0.
+ * r is the N of the down-projection MMA (M = 128 rows, N a multiple of 16 up to
+ * 256) and the K of the up-projection, which runs in steps of 32 (the last one
+ * half empty when r % 32 == 16). */
+LYNX_API int lynx_lora_rank_supported(int64_t r);
 
 /* ---- sizes ------------------------------------------------------------- */
 
@@ -93,8 +103,8 @@ LYNX_API size_t lynx_vals_bytes(int64_t M, int64_t K);
 LYNX_API size_t lynx_meta_bytes(int64_t M, int64_t K);
 
 /* Bytes of the workspace lynx_linear needs (kept values, metadata, row scales,
- * the bf16 LoRA down-projection [M,64], per-range partial sums, one
- * completion word per GEMM CTA, alignment). */
+ * the bf16 LoRA down-projection [M,r], per-range partial sums, one state word
+ * per 32-row slice, alignment).  r = 0 (no LoRA) sizes it as for r = 64. */
 LYNX_API size_t lynx_workspace_bytes(int64_t M, int64_t N, int64_t K, int64_t r);
 
 /* ---- the layer --------------------------------------------------------- */
@@ -150,12 +160,16 @@ LYNX_API int64_t lynx_sparsify_noalloc_max_rows(void);
 
 /* Y = S(X) W^T + bias + (X A^T) B^T  (S(X) = X when skip_sparsify != 0).
  *   X [M,K], W [N,K] (frozen backbone weight), bias [N] or NULL,
- *   A [r,K] and B [N,r] (LoRA, both or neither; r must be 64), Y [M,N] out.
+ *   A [r,K] and B [N,r] (LoRA, both or neither; r % 16 == 0, 16 <= r <= 256),
+ *   Y [M,N] out.
  *   workspace: caller-allocated device buffer of workspace_bytes >=
  *   lynx_workspace_bytes(M,N,K,r), used as scratch; at 256-byte aligned
  *   offsets, in this order, it ends up holding the kept values before
  *   compensation [M,K/2] bf16, the metadata, s per row [M] fp32 and T/s [M,r]
- *   bf16 (T = X A^T).
+ *   bf16 (T = X A^T).  The workspace needs no initial contents: every call
+ *   writes what it reads, the GEMM's per-row-block state words included (the
+ *   call's first kernel sets them to 0), so calls and replays of a captured
+ *   CUDA graph that reuse one workspace in stream order are independent.
  *   The compensation factor s is applied to the fp32 accumulator row, so
  *   Y = bf16(s * (S0 W^T + (T/s) B^T) + bias) with S0 the uncompensated kept
  *   values: the same product as S(X) W^T + T B^T with one rounding fewer. */
@@ -235,16 +249,20 @@ LYNX_API int lynx_linear_dense(const void* X, const void* W, const void* bias, c
 /* The sparse product on an S(X) made earlier by lynx_sparsify (or the
  * workspace of lynx_linear):  Y = S(X) W^T + bias + T B^T.
  *   vals [M,K/2] and meta as written by lynx_sparsify; T [M,r] bf16 or NULL,
- *   B [N,r] or NULL (both or neither, r = 64); other arguments as above. */
+ *   B [N,r] or NULL (both or neither, r as for lynx_linear); other arguments as
+ *   above. */
 LYNX_API int lynx_sparse_gemm(const void* vals, const void* meta, const void* T, const void* W,
                      const void* bias, const void* B, int64_t M, int64_t N, int64_t K, int64_t r,
                      void* Y, void* stream);
 
 /* ---- errors and metadata conversion ----------------------------------- */
 
-/* Synchronises `stream`, then reports (and clears) the current device's status
- * word: LYNX_ERR_DEVICE_TIMEOUT if a kernel gave up a bounded wait since the
- * last check, LYNX_ERR_CUDA if the stream holds a CUDA error, else LYNX_OK.
+/* Synchronises `stream`, then reports (and clears) the status word of that
+ * stream on the current device: LYNX_ERR_DEVICE_TIMEOUT if a kernel launched on
+ * it gave up a bounded wait since the last check, LYNX_ERR_CUDA if the stream
+ * holds a CUDA error, else LYNX_OK.  Errors of calls on other streams stay in
+ * their own words.  (A process uses at most 1023 words per device; the streams
+ * after those share one more word, which any of them reports and clears.)
  * *device_code (may be NULL) receives the raw device code (0 if none). */
 LYNX_API int lynx_check_error(void* stream, uint32_t* device_code);
 
@@ -264,6 +282,14 @@ LYNX_API int lynx_meta_canonical_to_hw(const uint8_t* canonical, uint8_t* hw, in
  * tail of the sparsify pass, so a call takes slightly longer.
  * Process-wide; returns the previous event. */
 LYNX_API void* lynx_profile_set_split_event(void* event);
+
+/* Profiling hook: part 1 makes lynx_linear (and lynx_linear_act) enqueue only
+ * its first kernel, the sparsify (or, on the dense path, LoRA-down) pass; part
+ * 2 only what follows it (the GEMM, after a reset of its per-row-block state
+ * words, and the split event, if set, between the two), on a workspace that
+ * an earlier full call filled.  0 (the default) runs the whole layer.
+ * Process-wide; returns the previous part (-1 for an invalid argument). */
+LYNX_API int lynx_profile_set_part(int part);
 
 /* Test hook (not for production use): when nonzero, kernels launched after
  * this call never load their inputs, so their bounded waits run out (about 2 s)

@@ -35,6 +35,37 @@ def test_status_strings(lib):
     assert lynx.lynx_lora_rank() == 64
 
 
+def test_lora_rank_rules(lib):
+    ok = [16, 32, 48, 64, 128, 240, 256]
+    bad = [0, 8, 24, 63, 65, 272, 512, -16]
+    assert all(lynx.lynx_lora_rank_supported(r) for r in ok)
+    assert not any(lynx.lynx_lora_rank_supported(r) for r in bad)
+    for r in ok:  # accepted by the checks; the call then fails only for want of a device
+        assert linear(lib, A=P, B=P, r=r) in (lynx.LYNX_ERR_CUDA, lynx.LYNX_OK), r
+    for r in bad:
+        assert linear(lib, A=P, B=P, r=r) == lynx.LYNX_ERR_UNSUPPORTED_SHAPE, r
+    # without A and B, r only sizes nothing: 0 or any supported rank
+    assert linear(lib, r=17) == lynx.LYNX_ERR_UNSUPPORTED_SHAPE
+
+
+@pytest.mark.parametrize("r", [16, 64, 256])
+def test_workspace_grows_with_rank(lib, r):
+    M, K = 4608, 3072
+    ws = lynx.lynx_workspace_bytes(M, 512, K, r)
+    # kept values, metadata, s, T [M,r] bf16, 8 split partials (sums and T),
+    # one state word per 32-row slice
+    floor = M * K + lynx.lynx_meta_bytes(M, K) + 4 * M + 2 * M * r + 8 * M * 8 + 8 * M * r * 4 + \
+        4 * -(-M // 32)
+    assert floor <= ws <= floor + 8 * 256
+
+
+def test_profile_part_hook(lib):
+    assert lynx.lynx_profile_set_part(1) == 0
+    assert lynx.lynx_profile_set_part(2) == 1
+    assert lib.lynx_profile_set_part(3) == -1
+    assert lynx.lynx_profile_set_part(0) == 2
+
+
 @pytest.mark.parametrize("M,K", [(1, 64), (128, 128), (129, 192), (4608, 3072), (4608, 12288)])
 def test_sizes(lib, M, K):
     assert lynx.lynx_vals_bytes(M, K) == M * K
@@ -63,7 +94,7 @@ def test_linear_argument_errors(lib):
     assert linear(lib, W=None) == lynx.LYNX_ERR_INVALID_ARG
     assert linear(lib, Y=None) == lynx.LYNX_ERR_INVALID_ARG
     assert linear(lib, A=P, B=None) == lynx.LYNX_ERR_INVALID_ARG
-    assert linear(lib, A=P, B=P, r=32) == lynx.LYNX_ERR_UNSUPPORTED_SHAPE
+    assert linear(lib, A=P, B=P, r=40) == lynx.LYNX_ERR_UNSUPPORTED_SHAPE
     assert linear(lib, K=100) == lynx.LYNX_ERR_UNSUPPORTED_SHAPE
     assert linear(lib, K=32) == lynx.LYNX_ERR_UNSUPPORTED_SHAPE
     assert linear(lib, N=12) == lynx.LYNX_ERR_UNSUPPORTED_SHAPE

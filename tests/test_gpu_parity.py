@@ -16,6 +16,7 @@ import oracle
 from activation_sparse_gemm_lynx_b200 import lynx, workloads
 
 import helpers
+import oracle_checks
 
 pytestmark = pytest.mark.gpu
 
@@ -193,12 +194,12 @@ def test_linear_is_deterministic():
     assert np.array_equal(y1, y2)
 
 
-def check_workspace(ws, inp, rows=None):
+def check_workspace(ws, inp, rows=None, r=64):
     """lynx_linear leaves in its workspace: the uncompensated kept values (exact
     copies of X), the metadata, s per row and T/s.  Checked on `rows`."""
     X = inp["X"]
     M, K = X.shape
-    vals, meta, scale, t = helpers.workspace_views(ws.cpu().numpy(), M, K)
+    vals, meta, scale, t = helpers.workspace_views(ws.cpu().numpy(), M, K, r)
     rows = np.arange(M) if rows is None else rows
     canon = helpers.canonical_from_hw(meta, M, K)[rows]
     ref = oracle.sparsify(X[rows])
@@ -206,6 +207,7 @@ def check_workspace(ws, inp, rows=None):
     assert np.array_equal(vals[rows], helpers.kept_from_x(X[rows], canon, K))
     assert np.allclose(scale[rows], ref["scale"], rtol=4e-6, atol=0)
     _, t_ref, _ = oracle.linear(X[rows], inp["W"][:8], None, inp["A"], inp["B"][:8])
+    assert t_ref.shape[1] == r
     s64 = ref["scale"].astype(np.float64)[:, None]
     t_over_s = t_ref / s64
     T = helpers.f32(t[rows]).astype(np.float64)
@@ -230,24 +232,112 @@ def test_workspace_holds_kept_values_scale_and_t():
 
 
 # ---------------------------------------------------------------------------
-# full-size workloads, in the launch configuration the benchmark times: sampled
-# rows against the oracle (rows are independent)
+# full-size workloads, in the launch configuration the benchmark times: Y on
+# every row against the oracle, the workspace (selection, kept values, s, T/s)
+# on sampled rows
 
 
 @pytest.mark.parametrize("name", ["attn_out", "mlp_up", "mlp_down"])
-def test_full_size_sampled_rows(name):
+def test_full_size_every_row(name):
     c = workloads.CONFIGS[name]
     inp = workloads.make_config_inputs(name)
     M, K = inp["X"].shape
+    ws = torch.empty(lynx.lynx_workspace_bytes(M, c.N, K, 64), dtype=torch.uint8, device=DEV)
+    args = [dev(inp[k]) for k in ("X", "W", "bias", "A", "B")]
+    Y = lynx.lynx_linear(*args, workspace=ws)
+    torch.cuda.synchronize()
+    st, code = lynx.lynx_check_error()
+    assert st == lynx.LYNX_OK, (st, code)
+    worst, fro = oracle_checks.linear_all_rows(host(Y), inp)
+    assert worst <= 1.0 and fro <= 5e-3, (name, worst, fro)
     rng = np.random.default_rng(99)
     rows = np.unique(np.concatenate([[0, 127, 128, M - 1], rng.choice(M, 28, replace=False)]))
-    ws = torch.empty(lynx.lynx_workspace_bytes(M, c.N, K, 64), dtype=torch.uint8, device=DEV)
-    check_linear(inp, rows=rows)
-    # S(X) of the sampled rows, from the same kind of call
-    args = [dev(inp[k]) for k in ("X", "W", "bias", "A", "B")]
-    lynx.lynx_linear(*args, workspace=ws)
-    torch.cuda.synchronize()
     check_workspace(ws, inp, rows=rows)
+
+
+# ---------------------------------------------------------------------------
+# the dense path's own entry point
+
+
+@pytest.mark.parametrize("M,N,K,lora", [
+    (300, 200, 576, True),     # 1-CTA GEMM, ragged
+    (512, 1024, 1024, True),   # CTA-pair GEMM, LoRA T combined inside the GEMM
+    (384, 768, 512, False),    # CTA-pair GEMM, no LoRA: one kernel
+])
+def test_linear_dense_entry_point(M, N, K, lora):
+    inp = workloads.make_linear_inputs(M, K, N, seed=M + N + K, lora=lora)
+    Y = lynx.lynx_linear_dense(*[dev(inp[k]) for k in ("X", "W", "bias", "A", "B")])
+    torch.cuda.synchronize()
+    st, code = lynx.lynx_check_error()
+    assert st == lynx.LYNX_OK, (st, code)
+    worst, fro = oracle_checks.linear_all_rows(host(Y), inp, skip=True)
+    assert worst <= 1.0 and fro <= 5e-3, (worst, fro)
+
+
+# ---------------------------------------------------------------------------
+# LoRA ranks other than the pages' 64: r % 16 == 0 up to 256 (r = 48 leaves the
+# last K = 32 step of the up-projection half empty)
+
+
+@pytest.mark.parametrize("r", [16, 48, 128, 256])
+@pytest.mark.parametrize("M,N,K", [(300, 200, 576), (512, 768, 1024)])
+@pytest.mark.parametrize("skip", [False, True])
+def test_linear_lora_ranks(r, M, N, K, skip):
+    inp = workloads.make_linear_inputs(M, K, N, r=r, seed=r * 7 + M)
+    ws = torch.empty(lynx.lynx_workspace_bytes(M, N, K, r), dtype=torch.uint8, device=DEV)
+    Y = lynx.lynx_linear(*[dev(inp[k]) for k in ("X", "W", "bias", "A", "B")], skip_sparsify=skip,
+                         workspace=ws)
+    torch.cuda.synchronize()
+    st, code = lynx.lynx_check_error()
+    assert st == lynx.LYNX_OK, (st, code)
+    worst, fro = oracle_checks.linear_all_rows(host(Y), inp, skip=skip)
+    assert worst <= 1.0 and fro <= 5e-3, (r, worst, fro)
+    if not skip:
+        _, _, _, t = helpers.workspace_views(ws.cpu().numpy(), M, K, r)
+        assert t.shape == (M, r)
+        check_workspace(ws, inp, rows=np.array([0, 1, M // 2, M - 1]), r=r)
+
+
+def test_garbage_workspace_and_stale_state_words():
+    """The workspace needs no initial contents: with every 32-bit word set to 2
+    (the 'combined' state of the GEMM's per-row-block words) and to -1, the
+    layer still matches the oracle, since each call clears those words first."""
+    inp = workloads.make_linear_inputs(512, 1024, 768, seed=21)
+    ws = torch.empty(lynx.lynx_workspace_bytes(512, 768, 1024, 64), dtype=torch.uint8, device=DEV)
+    args = [dev(inp[k]) for k in ("X", "W", "bias", "A", "B")]
+    for fill in (2, -1):
+        for skip in (False, True):
+            ws.view(torch.int32).fill_(fill)
+            Y = lynx.lynx_linear(*args, skip_sparsify=skip, workspace=ws)
+            torch.cuda.synchronize()
+            worst, fro = oracle_checks.linear_all_rows(host(Y), inp, skip=skip)
+            assert worst <= 1.0 and fro <= 5e-3, (fill, skip, worst, fro)
+    st, code = lynx.lynx_check_error()
+    assert st == lynx.LYNX_OK, (st, code)
+
+
+def test_layer_with_sms_held_by_another_stream():
+    """The CTA-pair GEMM needs no co-residency of its grid: while kernels on
+    other streams hold some SMs for about 20 ms, the layer at the mlp_up shape
+    (a full-device grid) completes without a timeout and matches the oracle."""
+    inp = workloads.make_config_inputs("mlp_up")
+    M = inp["X"].shape[0]
+    args = [dev(inp[k]) for k in ("X", "W", "bias", "A", "B")]
+    Y = lynx.lynx_linear(*args)  # one-time set-up outside the contended run
+    torch.cuda.synchronize()
+    side = [torch.cuda.Stream() for _ in range(6)]
+    cycles = 40_000_000  # about 20 ms at the B200's 1.965 GHz
+    for sstream in side:
+        with torch.cuda.stream(sstream):
+            torch.cuda._sleep(cycles)  # one block spinning for about 20 ms
+    Y.zero_()
+    lynx.lynx_linear(*args, Y=Y)
+    torch.cuda.synchronize()
+    st, code = lynx.lynx_check_error()
+    assert st == lynx.LYNX_OK, (st, code)
+    rows = np.unique(np.concatenate([[0, 1, 255, 256, M - 1], np.arange(7, M, 97)]))
+    worst, fro = oracle_checks.linear_all_rows(host(Y)[rows], inp, rows=rows)
+    assert worst <= 1.0 and fro <= 5e-3, (worst, fro)
 
 
 # ---------------------------------------------------------------------------
@@ -289,6 +379,30 @@ def test_device_timeout_in_the_fused_layer():
         lynx.lynx_debug_set_stall(False)
     assert st == lynx.LYNX_ERR_DEVICE_TIMEOUT and code != 0
     check_linear(inp)
+
+
+def test_device_timeout_stays_with_its_stream():
+    """A timeout raised by a call on one stream is reported by lynx_check_error
+    on that stream only; a call on another stream reports OK and is correct."""
+    inp = workloads.make_linear_inputs(256, 512, 256, seed=8)
+    args = [dev(inp[k]) for k in ("X", "W", "bias", "A", "B")]
+    a, b = torch.cuda.Stream(), torch.cuda.Stream()
+    lynx.lynx_debug_set_stall(True)
+    try:
+        with torch.cuda.stream(a):
+            lynx.lynx_linear(*args)
+    finally:
+        lynx.lynx_debug_set_stall(False)
+    with torch.cuda.stream(b):
+        Y = lynx.lynx_linear(*args)
+    st_b, code_b = lynx.lynx_check_error(b)
+    st_a, code_a = lynx.lynx_check_error(a)
+    assert st_b == lynx.LYNX_OK and code_b == 0
+    assert st_a == lynx.LYNX_ERR_DEVICE_TIMEOUT and code_a != 0
+    assert lynx.lynx_check_error(a) == (lynx.LYNX_OK, 0)
+    torch.cuda.synchronize()
+    worst, fro = oracle_checks.linear_all_rows(host(Y), inp)
+    assert worst <= 1.0 and fro <= 5e-3, (worst, fro)
 
 
 def check_selection_all_rows(inp, chunk=1024):

@@ -75,7 +75,8 @@ def test_graph_layers_match_oracle(sweep_and_plan):
         assert worst <= 1.0 and fro <= 5e-3, (plan[i][:2], worst, fro)
 
 
-@pytest.mark.parametrize("layer", [0, 3])  # qkv 3072->9216 and down 12288->3072 (GELU inputs)
+# qkv 3072->9216, out 3072->3072, up 3072->12288, down 12288->3072 (GELU inputs)
+@pytest.mark.parametrize("layer", [0, 1, 2, 3])
 @pytest.mark.parametrize("skip", [False, True])
 def test_full_size_sweep_layer_sampled_rows(layer, skip):
     """One linear of the sweep at its full size (M = 8192), in the launch
