@@ -67,6 +67,7 @@ constexpr uint32_t kBarCompute = 1;                   // named barrier of the ro
 // Every tile starts on a 1024-byte boundary (r % 16 == 0 makes r*128 a
 // multiple of 2048).
 struct SparsifyCtl {
+  uint32_t sel_table[64];      // selection code -> kept-pair byte selector | nibble << 16
   float2 half1[128];           // partial sums of the second half of each row
   uint64_t full[kStages];
   uint64_t empty[kStages];     // row threads done with a stage (one arrival per warp)
@@ -100,46 +101,74 @@ __host__ __device__ inline uint32_t lora_tmem_cols(int r) {
   return c;
 }
 
-// acc_lo += |low bf16 of w|, acc_hi += |high bf16 of w|: each half widened to
-// fp32 exactly, the magnitude taken by the add's operand modifier
-__device__ __forceinline__ void add_abs_pair(float& acc_lo, float& acc_hi, uint32_t w) {
-  acc_lo = __fadd_rn(acc_lo, fabsf(__uint_as_float(w << 16)));
-  acc_hi = __fadd_rn(acc_hi, fabsf(__uint_as_float(w & 0xFFFF0000u)));
+// acc_lo += low bf16 of w, acc_hi += high bf16 of w, in fp32 (one rounding
+// each; the bf16 operand is exact in fp32)
+__device__ __forceinline__ void add_bf16_pair(float& acc_lo, float& acc_hi, uint32_t w) {
+  asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %2;\n\t"
+      "add.rn.f32.bf16 %0, lo, %0;\n\tadd.rn.f32.bf16 %1, hi, %1;\n\t}"
+      : "+f"(acc_lo), "+f"(acc_hi)
+      : "r"(w));
+}
+
+// per 16-bit lane: 0xFFFF if a >= b, else 0 (bf16 compare; for the
+// non-negative finite magnitudes used here the order of the bit patterns)
+__device__ __forceinline__ uint32_t ge_bf16x2(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("set.ge.u32.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+
+// The selection of a group of 4 is decided by the six comparisons
+// "x_i beats x_j" (i < j): |x_i| >= |x_j|, so a tie goes to the lower index.
+// They come out of three bf16x2 compares as a 6-bit code,
+//   bit 0: |x0| >= |x2|   bit 1: |x0| >= |x3|   bit 2: |x0| >= |x1|
+//   bit 3: |x1| >= |x3|   bit 4: |x1| >= |x2|   bit 5: |x2| >= |x3|,
+// and a 64-entry table gives, per code, the byte selector that packs the two
+// kept values (lower position in the low half) and the nibble lo | hi << 2.
+// Value i is kept when fewer than two values beat it; a code that no order of
+// four magnitudes produces maps to the two least beaten values.
+__device__ __forceinline__ uint32_t selection_table_entry(uint32_t code) {
+  const int p02 = code & 1, p03 = (code >> 1) & 1, p01 = (code >> 2) & 1;
+  const int p13 = (code >> 3) & 1, p12 = (code >> 4) & 1, p23 = (code >> 5) & 1;
+  const int beaten[4] = {(1 - p01) + (1 - p02) + (1 - p03), p01 + (1 - p12) + (1 - p13),
+                         p02 + p12 + (1 - p23), p03 + p13 + p23};
+  int lo = -1, hi = -1;
+  for (int limit = 0; limit <= 3 && hi < 0; ++limit)  // the least beaten first, lower index first
+    for (int i = 0; i < 4 && hi < 0; ++i)
+      if (beaten[i] == limit && i != lo) {
+        if (lo < 0) lo = i;
+        else hi = i;
+      }
+  if (hi < lo) {
+    const int t = lo;
+    lo = hi;
+    hi = t;
+  }
+  const uint32_t sel = (2u * lo) | ((2u * lo + 1u) << 4) | ((2u * hi) << 8) | ((2u * hi + 1u) << 12);
+  return sel | ((static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 2)) << 16);
 }
 
 // Top-2 of the 4 bf16 values in (w0 = x1:x0, w1 = x3:x2) by magnitude, ties to
-// the lower index, together with the group's terms of the row's L1 sum.  Each
-// value is widened to fp32 (exact); its magnitude bits with (3 - i) in the two
-// lowest bits form a distinct key, so a larger key is a larger magnitude or, on
-// equal magnitude, a lower index, and the two largest keys come out of a
-// 4-input max/min network.  Adds |x0|, |x2| to la_even and |x1|, |x3| to
-// la_odd; returns the nibble lo | hi << 2 and the kept pair packed (x_lo in the
-// low half).
-__device__ __forceinline__ uint32_t select_group(uint32_t w0, uint32_t w1, uint32_t& kept,
-                                                 float& la_even, float& la_odd) {
-  const uint32_t f0 = w0 << 16, f1 = w0 & 0xFFFF0000u;
-  const uint32_t f2 = w1 << 16, f3 = w1 & 0xFFFF0000u;
-  la_even = __fadd_rn(la_even, fabsf(__uint_as_float(f0)));
-  la_odd = __fadd_rn(la_odd, fabsf(__uint_as_float(f1)));
-  la_even = __fadd_rn(la_even, fabsf(__uint_as_float(f2)));
-  la_odd = __fadd_rn(la_odd, fabsf(__uint_as_float(f3)));
-  // the 15 magnitude bits go to bits 17..31 by a multiply that drops the sign
-  // (the FMA pipe, not the busier ALU pipe); the low 17 bits of each product
-  // are zero, so 3 - i fits below them
-  const uint32_t k0 = w0 * 131072u + 3u;
-  const uint32_t k1 = f1 * 2u + 2u;
-  const uint32_t k2 = w1 * 131072u + 1u;
-  const uint32_t k3 = f3 * 2u;
-  const uint32_t p = max(k0, k1), q = min(k0, k1);
-  const uint32_t r = max(k2, k3), u = min(k2, k3);
-  const uint32_t t1 = max(p, r);
-  const uint32_t t2 = max(min(p, r), max(q, u));
-  const uint32_t a = t1 & 3u, b = t2 & 3u;  // 3 - index of the two winners
-  const uint32_t mx = max(a, b), mn = min(a, b);  // lo = 3 - mx, hi = 3 - mn
-  // byte selector picking elements lo and hi out of the 8 bytes (w1:w0):
-  // 0x1010 + lo * 0x22 + hi * 0x2200, with the constant parts folded
-  kept = __byte_perm(w0, w1, 0x7676u - mx * 0x22u - mn * 0x2200u);
-  return 15u - mx - mn * 4u;  // lo | hi << 2
+// the lower index, together with the group's terms of the row's two L1 sums:
+// |x0|, |x2| to la_even and |x1|, |x3| to la_odd, the kept magnitudes to lk_lo
+// and lk_hi.  Returns the nibble lo | hi << 2 and the kept pair packed (x_lo in
+// the low half).
+__device__ __forceinline__ uint32_t select_group(uint32_t w0, uint32_t w1, const uint32_t* table,
+                                                 uint32_t& kept, float& la_even, float& la_odd,
+                                                 float& lk_lo, float& lk_hi) {
+  const uint32_t a0 = w0 & 0x7FFF7FFFu;  // |x1| : |x0|
+  const uint32_t a1 = w1 & 0x7FFF7FFFu;  // |x3| : |x2|
+  add_bf16_pair(la_even, la_odd, a0);
+  add_bf16_pair(la_even, la_odd, a1);
+  const uint32_t c1 = ge_bf16x2(a0, a1);                                // x0>=x2 | x1>=x3
+  const uint32_t c2 = ge_bf16x2(a0, __byte_perm(a1, 0, 0x1032));        // x0>=x3 | x1>=x2
+  const uint32_t c3 = ge_bf16x2(__byte_perm(a0, a1, 0x5410), __byte_perm(a0, a1, 0x7632));  // x0>=x1 | x2>=x3
+  uint32_t code = (c1 & 0x00010001u) | (c2 & 0x00020002u) | (c3 & 0x00040004u);
+  code = (code | (code >> 13)) & 0x3Fu;
+  const uint32_t ent = table[code];
+  kept = __byte_perm(w0, w1, ent);
+  add_bf16_pair(lk_lo, lk_hi, __byte_perm(a0, a1, ent));
+  return ent >> 16;
 }
 
 __device__ __forceinline__ uint32_t scale_pair(uint32_t w, float s) {
@@ -187,6 +216,7 @@ sparsify_kernel(const __grid_constant__ SparsifyLaunch p) {
     sm.abort_flag = 0u;
     fence_mbar_init();
   }
+  if (threadIdx.x >= 64 && threadIdx.x < 128) sm.sel_table[threadIdx.x - 64] = selection_table_entry(threadIdx.x - 64);
   // The first box's loads leave before the rest of the prologue (TMEM
   // allocation, the block barrier): its latency is the one nothing else hides.
   // The other stages' loads follow only once it has landed, so that the first
@@ -365,16 +395,15 @@ sparsify_kernel(const __grid_constant__ SparsifyLaunch p) {
       const uint4 v2 = *reinterpret_cast<const uint4*>(tile + ld_off2);
       const uint4 v3 = *reinterpret_cast<const uint4*>(tile + ld_off3);
       uint32_t kw[8];
-      const uint32_t n0 = select_group(v0.x, v0.y, kw[0], la0, la1);
-      const uint32_t n1 = select_group(v0.z, v0.w, kw[1], la0, la1);
-      const uint32_t n2 = select_group(v1.x, v1.y, kw[2], la0, la1);
-      const uint32_t n3 = select_group(v1.z, v1.w, kw[3], la0, la1);
-      const uint32_t n4 = select_group(v2.x, v2.y, kw[4], la0, la1);
-      const uint32_t n5 = select_group(v2.z, v2.w, kw[5], la0, la1);
-      const uint32_t n6 = select_group(v3.x, v3.y, kw[6], la0, la1);
-      const uint32_t n7 = select_group(v3.z, v3.w, kw[7], la0, la1);
-#pragma unroll
-      for (int i = 0; i < 8; ++i) add_abs_pair(lk0, lk1, kw[i]);
+      const uint32_t* tab = sm.sel_table;
+      const uint32_t n0 = select_group(v0.x, v0.y, tab, kw[0], la0, la1, lk0, lk1);
+      const uint32_t n1 = select_group(v0.z, v0.w, tab, kw[1], la0, la1, lk0, lk1);
+      const uint32_t n2 = select_group(v1.x, v1.y, tab, kw[2], la0, la1, lk0, lk1);
+      const uint32_t n3 = select_group(v1.z, v1.w, tab, kw[3], la0, la1, lk0, lk1);
+      const uint32_t n4 = select_group(v2.x, v2.y, tab, kw[4], la0, la1, lk0, lk1);
+      const uint32_t n5 = select_group(v2.z, v2.w, tab, kw[5], la0, la1, lk0, lk1);
+      const uint32_t n6 = select_group(v3.x, v3.y, tab, kw[6], la0, la1, lk0, lk1);
+      const uint32_t n7 = select_group(v3.z, v3.w, tab, kw[7], la0, la1, lk0, lk1);
       meta_ptr[0] = static_cast<uint16_t>(n0 + n1 * 16u + n2 * 256u + n3 * 4096u);
       meta_ptr[64] = static_cast<uint16_t>(n4 + n5 * 16u + n6 * 256u + n7 * 4096u);
       meta_ptr += meta_hi_half ? 1020 : 4;
