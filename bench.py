@@ -41,7 +41,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # GEMM's sources at the capture: the bench reports the figure only while the
 # sources still hash the same, else null ("stale").
 GEMM_SOURCES = ("gemm_pair_kernel.cu", "lynx_ptx.cuh", "lynx_internal.h", "lynx_act.cuh")
-GEMM_DRAM_TRAFFIC = {}
+GEMM_DRAM_TRAFFIC = {"mlp_up": {"bytes": 103.165e6 + 82.323e6, "src": "82e9d7345104", "captured": "2026-12-03"}}
 
 def uses_pair_gemm(M, N, K):
     """The library's choice: the CTA-pair GEMM unless the shape cannot feed it."""
