@@ -79,6 +79,9 @@ def parse_args(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-per-config", action="store_true",
                     help="skip the per_config block (the other DiT shapes)")
+    ap.add_argument("--gather-y", action="store_true",
+                    help="with --gpus N > 1: also time the layer followed by an all-gather of Y "
+                         "(every rank ends with all N x M rows), reported as y_gather")
     ap.add_argument("--only-linear", action="store_true",
                     help="time the layer only (no comparisons, e2e or CPU baseline); "
                          "the short launch sequence used for ncu captures")
@@ -600,6 +603,21 @@ def run_lynx(args):
         result["speedup_vs_unfused_act"] = unfused_ms / ms_step
         result["breakdown_ms"]["linear_then_separate_act"] = unfused_ms
         result["dense_note"] = "torch.matmul then torch GELU (tanh) as a separate pass"
+
+    if args.gather_y and world > 1:
+        # the row-sharded layer followed by an NCCL all-gather of Y's row blocks
+        from activation_sparse_gemm_lynx_b200 import sharded
+
+        def step_gather():
+            lt.step_linear()
+            sharded.gather_rows(lt.Y, world * M)
+
+        for _ in range(3):
+            step_gather()
+        g_ms = max_over_ranks(statistics.mean(lt.timed(step_gather, ncmp)), world)
+        result["y_gather"] = {"ms_per_step": g_ms, "value": aggregate_tflops(flops, g_ms, world),
+                              "unit": "TFLOP/s", "gathered_bytes_per_rank": 2 * M * N * (world - 1),
+                              "note": "lynx_linear on each rank's rows, then all_gather_into_tensor of Y"}
 
     # the other DiT shapes of the same targets, measured in this run the same
     # way (fewer steps); the headline stays the selected workload
