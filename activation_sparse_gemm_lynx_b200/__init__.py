@@ -5,7 +5,7 @@
 S(X) keeps, per token row, the 2 largest magnitudes of every 4 consecutive
 values (ties to the lower position), rescaled by the fp32 norm-compensation
 factor sum|x| / sum|kept| and rounded to bf16; the product runs on sparse
-tensor cores (tcgen05.mma.sp) and the rank-64 LoRA residual on the dense X
+tensor cores (tcgen05.mma.sp) and the rank-r LoRA residual on the dense X
 plus the bias are added in the same accumulator before one bf16 store.
 
 The public entry points mirror the C ABI of ``include/lynx.h``; see
@@ -21,13 +21,16 @@ from .lynx import (  # noqa: F401
     lynx_linear,
     lynx_linear_act,
     lynx_linear_dense,
+    lynx_linear_fused,
     lynx_linear_host,
     lynx_linear_host_act,
     lynx_linear_host_workspace_bytes,
     lynx_lora_rank,
+    lynx_lora_rank_supported,
     lynx_meta_bytes,
     lynx_meta_canonical_to_hw,
     lynx_meta_hw_to_canonical,
+    lynx_profile_set_part,
     lynx_profile_set_split_event,
     lynx_sparse_gemm,
     lynx_sparsify,

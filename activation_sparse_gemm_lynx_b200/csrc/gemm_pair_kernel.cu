@@ -34,6 +34,7 @@
 #include "lynx_act.cuh"
 #include "lynx_internal.h"
 #include "lynx_ptx.cuh"
+#include "lynx_select.cuh"
 
 namespace lynx {
 
@@ -56,13 +57,19 @@ constexpr uint16_t kPairMask = 0x3;
 // path (8 MMAs per hand-off instead of 4); on the sparse path 4 stages of 4 MMAs
 // beat 2 stages of 8.  LoRA stages (K = 32 each) reuse the A / B slots with
 // 64-byte-row tiles.
-template <bool SPARSE>
+// FUSED (sparse): the stage holds the dense X tile (two 128 x 64 tiles); the
+// epilogue warps compress it in place into the first one, which is then the
+// MMA's A operand, and write the metadata block.
+template <bool SPARSE, bool FUSED = false>
 struct PairCfg {
   static constexpr int kBK = 128;
   static constexpr uint32_t kABytes = SPARSE ? 128u * 128u : 2u * 128u * 128u;  // own 128 rows
+  static constexpr uint32_t kXBytes = FUSED ? 2u * 128u * 128u : 0u;  // dense X tile (fused)
+  static constexpr uint32_t kBOff = FUSED ? kXBytes : kABytes;        // W tile
   static constexpr uint32_t kBBytes = 128u * static_cast<uint32_t>(kBK) * 2u;  // own 128 W rows
+  static constexpr uint32_t kEOff = kBOff + kBBytes;                   // metadata block
   static constexpr uint32_t kEBytes = SPARSE ? 2048u : 0u;
-  static constexpr uint32_t kStageBytes = ((kABytes + kBBytes + kEBytes + 1023u) / 1024u) * 1024u;
+  static constexpr uint32_t kStageBytes = ((kEOff + kEBytes + 1023u) / 1024u) * 1024u;
   // of the 227 KB: 16 KB epilogue store staging, ~3 KB barriers / bias / alignment
   static constexpr int kStagesFit = static_cast<int>((208u * 1024u) / kStageBytes);
   static constexpr int kStages = kStagesFit > 8 ? 8 : kStagesFit;
@@ -71,11 +78,12 @@ struct PairCfg {
   static constexpr uint32_t kLoraBBytes = 128u * 64u;  // B: own 128 rows x 32
   static_assert(kStages >= 3, "pipeline too shallow");
   static_assert(kBarStage0 + kStages <= 16, "named barriers");
+  static_assert(!FUSED || SPARSE, "the fused variant is sparse");
 };
 
-template <bool SPARSE>
+template <bool SPARSE, bool FUSED = false>
 struct __align__(1024) PairSmem {
-  using C = PairCfg<SPARSE>;
+  using C = PairCfg<SPARSE, FUSED>;
   uint8_t stage[C::kStages][C::kStageBytes];
   uint8_t ystage[8][2][1024];  // per epilogue warp: two 32 rows x 16 columns bf16 tiles (32B swizzle)
   uint64_t full[C::kStages];   // used in the leader CTA
@@ -84,6 +92,9 @@ struct __align__(1024) PairSmem {
   uint64_t acc_empty;          // used in the leader CTA (both CTAs' epilogues arrive)
   uint64_t drain;
   uint64_t rows_ready;         // the rows of T of all this CTA's tiles are combined (fused, LoRA)
+  uint64_t xfull[C::kStages];  // FUSED: this CTA's X tile of the stage has landed
+  uint64_t afull[C::kStages];  // FUSED (leader): both CTAs' compressed A and metadata are written
+  uint32_t sel_table[64];      // FUSED: selection code -> kept-pair byte selector | nibble << 16
   float bias_s[256];
   uint32_t tmem_base;
   uint32_t own_claimed[32];    // fused combining: which of the CTA's own slices it claimed
@@ -277,12 +288,68 @@ __device__ __noinline__ bool ensure_rows_of_tiles(const GemmLaunch& p, Smem& sm,
   }
 }
 
-template <bool SPARSE, int ACT>
+// FUSED: the epilogue warps turn the dense X tile of each main stage of one
+// tile into the MMA's sparse operand, in place, and tell the leader (afull):
+// thread et takes row et / 2 and half et % 2 of the stage's 128 K (16 groups of
+// 4).  The compressed row (64 kept values) goes to the row's 128 bytes of the
+// first X tile, in its 128-byte swizzle, which is the A layout of the sparse
+// path; the nibbles go to the stage's metadata block in the operand layout of
+// tcgen05.mma.sp (the same as the sparsify pass writes).  The two threads of a
+// row are neighbouring lanes, and a warp reads all its X before it writes.
+// LoRA stages only pass the barrier on.  `g` is the stage counter shared with
+// the producer and the MMA issuer.  Returns false if a wait ran out (this
+// warp's answer; the caller makes it common).
+template <typename C, typename Smem>
+__device__ __forceinline__ bool compress_tile_stages(Smem& sm, uint32_t& g, int nk, int steps, uint32_t et,
+                                                     uint32_t lane) {
+  const uint32_t r = et >> 1, h = et & 1u, sw = r & 7u;
+  for (int kit = 0; kit < steps; ++kit, ++g) {
+    const uint32_t slot = g % C::kStages;
+    const uint32_t ph = (g / C::kStages) & 1u;
+    bool ok = !sm.abort_flag && mbar_wait(&sm.xfull[slot], ph);
+    if (!__all_sync(0xffffffffu, ok)) return false;
+    if (kit < nk) {
+      uint8_t* st = sm.stage[slot];
+      const uint8_t* xrow = st + h * 16384u + r * 128u;
+      uint4 v[8];
+#pragma unroll
+      for (int c = 0; c < 8; ++c) v[c] = *reinterpret_cast<const uint4*>(xrow + ((c ^ sw) << 4));
+      uint32_t kept[16], nib[16];
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        nib[2 * c] = select_group_kept(v[c].x, v[c].y, sm.sel_table, kept[2 * c]);
+        nib[2 * c + 1] = select_group_kept(v[c].z, v[c].w, sm.sel_table, kept[2 * c + 1]);
+      }
+      __syncwarp();  // the whole warp has read its X rows before any is overwritten
+      uint8_t* arow = st + r * 128u;
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        *reinterpret_cast<uint4*>(arow + (((4u * h + i) ^ sw) << 4)) =
+            make_uint4(kept[4 * i], kept[4 * i + 1], kept[4 * i + 2], kept[4 * i + 3]);
+      // 16-bit field of (row r, 16-K chunk c16): lane (r%8) + 8(c16%2) + 16(r/16),
+      // 32-bit word c16/2, upper half for rows with (r/8) odd
+      uint16_t* e = reinterpret_cast<uint16_t*>(st + C::kEOff);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const uint32_t c16 = 4u * h + i;
+        const uint32_t tl = (r & 7u) + 8u * (c16 & 1u) + 16u * (r >> 4);
+        e[tl * 8u + (c16 >> 1) * 2u + ((r >> 3) & 1u)] =
+            static_cast<uint16_t>(nib[4 * i] + nib[4 * i + 1] * 16u + nib[4 * i + 2] * 256u + nib[4 * i + 3] * 4096u);
+      }
+      fence_proxy_async_smem();  // the MMA reads them through the async proxy
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive_cluster_release(mapa_shared(smem_u32(&sm.afull[slot]), 0));
+  }
+  return true;
+}
+
+template <bool SPARSE, int ACT, bool FUSED>
 __global__ void __launch_bounds__(kThreads, 1)
 lynx_gemm_pair_kernel(const __grid_constant__ GemmLaunch p) {
-  using C = PairCfg<SPARSE>;
+  using C = PairCfg<SPARSE, FUSED>;
   extern __shared__ uint8_t smem_raw[];
-  PairSmem<SPARSE>& sm = *reinterpret_cast<PairSmem<SPARSE>*>(
+  PairSmem<SPARSE, FUSED>& sm = *reinterpret_cast<PairSmem<SPARSE, FUSED>*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
 
   const uint32_t warp = warp_id_sync();
@@ -310,9 +377,17 @@ lynx_gemm_pair_kernel(const __grid_constant__ GemmLaunch p) {
     mbar_init(&sm.acc_empty, 2 * 8);
     mbar_init(&sm.drain, 1);
     mbar_init(&sm.rows_ready, 1);
+    if (FUSED) {
+      for (int s = 0; s < C::kStages; ++s) {
+        mbar_init(&sm.xfull[s], 1);
+        mbar_init(&sm.afull[s], 2 * 8);  // the 8 epilogue warps of both CTAs
+      }
+    }
     sm.abort_flag = 0u;
     fence_mbar_init();
   }
+  if (FUSED && threadIdx.x >= 64 && threadIdx.x < 128)
+    sm.sel_table[threadIdx.x - 64] = selection_table_entry(threadIdx.x - 64);
   if (warp == 1) {
     tmem_alloc_pair(&sm.tmem_base, kTmemCols);
     tmem_relinquish_pair();
@@ -357,7 +432,16 @@ lynx_gemm_pair_kernel(const __grid_constant__ GemmLaunch p) {
           }
           uint8_t* st = sm.stage[slot];
           const uint32_t lead_full = mapa_shared(smem_u32(&sm.full[slot]), 0);
-          if (kit < nk) {
+          if (FUSED && kit < nk) {
+            // this CTA's dense X tile into its own shared memory (own barrier);
+            // the W tile as on the sparse path
+            mbar_arrive_expect_tx(&sm.xfull[slot], C::kXBytes);
+            tma_load_2d(st, &p.tm_a, &sm.xfull[slot], kit * C::kBK, row0);
+            tma_load_2d(st + 16384, &p.tm_a, &sm.xfull[slot], kit * C::kBK + 64, row0);
+            if (leader) mbar_arrive_expect_tx(&sm.full[slot], 2u * C::kBBytes);
+            tma_load_2d_pair(st + C::kBOff, &p.tm_b, lead_full, kit * C::kBK, col0);
+            tma_load_2d_pair(st + C::kBOff + 16384, &p.tm_b, lead_full, kit * C::kBK + 64, col0);
+          } else if (kit < nk) {
             if (leader) mbar_arrive_expect_tx(&sm.full[slot], 2u * (C::kABytes + C::kBBytes + C::kEBytes));
             // A: 64 kept values (sparse) or 64 dense values (dense) per row
             if (SPARSE) {
@@ -366,12 +450,11 @@ lynx_gemm_pair_kernel(const __grid_constant__ GemmLaunch p) {
               tma_load_2d_pair(st, &p.tm_a, lead_full, kit * C::kBK, row0);
               tma_load_2d_pair(st + 16384, &p.tm_a, lead_full, kit * C::kBK + 64, row0);
             }
-            tma_load_2d_pair(st + C::kABytes, &p.tm_b, lead_full, kit * C::kBK, col0);
-            tma_load_2d_pair(st + C::kABytes + 16384, &p.tm_b, lead_full, kit * C::kBK + 64, col0);
+            tma_load_2d_pair(st + C::kBOff, &p.tm_b, lead_full, kit * C::kBK, col0);
+            tma_load_2d_pair(st + C::kBOff + 16384, &p.tm_b, lead_full, kit * C::kBK + 64, col0);
             if (SPARSE) {
               // metadata block (mb, kit): 2 KB seen as 8 rows of 256 bytes
-              tma_load_2d_pair(st + C::kABytes + C::kBBytes, &p.tm_e, lead_full, 0,
-                               (mb * kblocks + kit) * 8);
+              tma_load_2d_pair(st + C::kEOff, &p.tm_e, lead_full, 0, (mb * kblocks + kit) * 8);
             }
           } else {
             const int l = kit - nk;
@@ -393,10 +476,19 @@ lynx_gemm_pair_kernel(const __grid_constant__ GemmLaunch p) {
               asm volatile("fence.proxy.async.global;" ::: "memory");  // T is then read by TMA
               rows_ready = true;
             }
+            if (FUSED) mbar_arrive(&sm.xfull[slot]);  // no X in a LoRA stage: the phase just passes
             if (leader) mbar_arrive_expect_tx(&sm.full[slot], 2u * (C::kLoraABytes + C::kLoraBBytes));
             tma_load_2d_pair(st, &p.tm_t, lead_full, l * 32, row0);
-            tma_load_2d_pair(st + C::kABytes, &p.tm_lb, lead_full, l * 32, col0);
+            tma_load_2d_pair(st + C::kBOff, &p.tm_lb, lead_full, l * 32, col0);
           }
+        }
+      }
+      // fused: this CTA's last X loads have landed (normally already consumed)
+      if (FUSED) {
+        for (uint32_t b = g; b > 0 && b + C::kStages > g; --b) {
+          const uint32_t x = b - 1;
+          if (!mbar_wait(&sm.xfull[x % C::kStages], (x / C::kStages) & 1u, kWaitLimitNs / 4))
+            record_error(p.status, kDevTimeoutDrain);
         }
       }
       // drain (leader): the last fill of every stage, both CTAs' bytes, has landed
@@ -439,11 +531,11 @@ lynx_gemm_pair_kernel(const __grid_constant__ GemmLaunch p) {
           }
           tc_fence_after();
           const uint32_t sa = smem_u32(sm.stage[slot]);
-          const uint32_t sb = sa + C::kABytes;
+          const uint32_t sb = sa + C::kBOff;
           if (kit < nk) {
             if (SPARSE) {
               eslot = (eslot + 1) % kEslots;
-              const uint64_t edesc = make_sdesc(sb + C::kBBytes, 2048, 128, kSwNone);
+              const uint64_t edesc = make_sdesc(sa + C::kEOff, 2048, 128, kSwNone);
               if (elect_one()) tc_cp_128x128b_pair(sm.tmem_base + C::kEcol0 + 4 * eslot, edesc);
               __syncwarp();
 #pragma unroll
@@ -504,6 +596,8 @@ lynx_gemm_pair_kernel(const __grid_constant__ GemmLaunch p) {
           const uint32_t slot = g % C::kStages;
           const uint32_t ph = (g / C::kStages) & 1u;
           bool ok = !sm.abort_flag && mbar_wait(&sm.full[slot], ph);
+          // fused: both CTAs' epilogue warps have compressed this stage's X
+          if (FUSED) ok = ok && !sm.abort_flag && mbar_wait_cluster(&sm.afull[slot], ph);
           ok = __all_sync(0xffffffffu, ok);
           if (!ok && lane == 0 && !sm.abort_flag) {
             record_error(p.status, kDevTimeoutFull);
@@ -537,7 +631,18 @@ lynx_gemm_pair_kernel(const __grid_constant__ GemmLaunch p) {
       if (et == 0 && lora) mbar_arrive(&sm.rows_ready);  // the producer may load T
     }
     int acc_count = 0;
+    uint32_t g_fused = 0;  // FUSED: the stage counter of the compression
     for (int tile = cluster_id; tile < ntiles; tile += nclusters, ++acc_count) {
+      if (FUSED) {
+        const bool ok = compress_tile_stages<C>(sm, g_fused, nk, steps, et, lane);
+        if (named_bar_red_or(kBarEpilogue, kEpiThreads, !ok)) {
+          if (et == 0 && !sm.abort_flag) {
+            record_error(p.status, kDevTimeoutFull);
+            sm.abort_flag = 1u;
+          }
+          break;
+        }
+      }
       int pm, nb;
       pair_tile_coords(tile, ntm2, ntn, p.group_m, pm, nb);
       const int64_t grow = static_cast<int64_t>(pm) * 256 + rank * 128 + row;
@@ -618,22 +723,28 @@ lynx_gemm_pair_kernel(const __grid_constant__ GemmLaunch p) {
   if (warp == 1) tmem_dealloc_pair(sm.tmem_base, kTmemCols);
 }
 
-template <bool SPARSE, int ACT>
+// the opt-in limit of dynamic shared memory per block on sm_100 (227 KB), with
+// the 1 KB the kernel spends on aligning its base
+static_assert(sizeof(PairSmem<true, false>) + 1024 <= 232448, "sparse pair GEMM shared memory");
+static_assert(sizeof(PairSmem<false, false>) + 1024 <= 232448, "dense pair GEMM shared memory");
+static_assert(sizeof(PairSmem<true, true>) + 1024 <= 232448, "fused pair GEMM shared memory");
+
+template <bool SPARSE, int ACT, bool FUSED>
 cudaError_t configure_pair_variant() {
   static std::once_flag once[64];
   static cudaError_t configured[64];
   return once_per_device(once, configured, []() {
-    return cudaFuncSetAttribute(lynx_gemm_pair_kernel<SPARSE, ACT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                static_cast<int>(sizeof(PairSmem<SPARSE>) + 1024));
+    return cudaFuncSetAttribute(lynx_gemm_pair_kernel<SPARSE, ACT, FUSED>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                static_cast<int>(sizeof(PairSmem<SPARSE, FUSED>) + 1024));
   });
 }
 
-template <bool SPARSE, int ACT>
+template <bool SPARSE, int ACT, bool FUSED>
 cudaLaunchConfig_t pair_config(int grid, cudaStream_t stream, cudaLaunchAttribute (&attr)[2]) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
   cfg.blockDim = dim3(kThreads, 1, 1);
-  cfg.dynamicSmemBytes = sizeof(PairSmem<SPARSE>) + 1024;
+  cfg.dynamicSmemBytes = sizeof(PairSmem<SPARSE, FUSED>) + 1024;
   cfg.stream = stream;
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
@@ -646,16 +757,16 @@ cudaLaunchConfig_t pair_config(int grid, cudaStream_t stream, cudaLaunchAttribut
   return cfg;
 }
 
-template <bool SPARSE, int ACT>
+template <bool SPARSE, int ACT, bool FUSED>
 cudaError_t launch_pair_variant(const GemmLaunch& p, cudaStream_t stream) {
-  cudaError_t e = configure_pair_variant<SPARSE, ACT>();
+  cudaError_t e = configure_pair_variant<SPARSE, ACT, FUSED>();
   if (e != cudaSuccess) return e;
   cudaLaunchAttribute attr[2];
-  cudaLaunchConfig_t cfg = pair_config<SPARSE, ACT>(p.grid, stream, attr);
-  return cudaLaunchKernelEx(&cfg, lynx_gemm_pair_kernel<SPARSE, ACT>, p);
+  cudaLaunchConfig_t cfg = pair_config<SPARSE, ACT, FUSED>(p.grid, stream, attr);
+  return cudaLaunchKernelEx(&cfg, lynx_gemm_pair_kernel<SPARSE, ACT, FUSED>, p);
 }
 
-template <bool SPARSE, int ACT>
+template <bool SPARSE, int ACT, bool FUSED>
 int pair_max_clusters_variant() {
   static std::once_flag once[64];
   static int clusters[64];
@@ -663,12 +774,12 @@ int pair_max_clusters_variant() {
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
   std::call_once(once[dev], [dev]() {
     clusters[dev] = 0;
-    if (configure_pair_variant<SPARSE, ACT>() != cudaSuccess) return;
+    if (configure_pair_variant<SPARSE, ACT, FUSED>() != cudaSuccess) return;
     cudaLaunchAttribute attr[2];
-    cudaLaunchConfig_t cfg = pair_config<SPARSE, ACT>(2, nullptr, attr);
+    cudaLaunchConfig_t cfg = pair_config<SPARSE, ACT, FUSED>(2, nullptr, attr);
     cfg.numAttrs = 1;  // the cluster shape is what matters here
     int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, lynx_gemm_pair_kernel<SPARSE, ACT>, &cfg) == cudaSuccess)
+    if (cudaOccupancyMaxActiveClusters(&n, lynx_gemm_pair_kernel<SPARSE, ACT, FUSED>, &cfg) == cudaSuccess)
       clusters[dev] = n;
     else
       (void)cudaGetLastError();  // a failed query is not sticky; the caller falls back
@@ -678,18 +789,25 @@ int pair_max_clusters_variant() {
 
 }  // namespace
 
-int gemm_pair_max_clusters(bool sparse, int act) {
+int gemm_pair_max_clusters(bool sparse, int act, bool fused) {
+  if (fused)
+    return act == kActGeluTanh ? pair_max_clusters_variant<true, kActGeluTanh, true>()
+                               : pair_max_clusters_variant<true, kActNone, true>();
   if (act == kActGeluTanh)
-    return sparse ? pair_max_clusters_variant<true, kActGeluTanh>() : pair_max_clusters_variant<false, kActGeluTanh>();
-  return sparse ? pair_max_clusters_variant<true, kActNone>() : pair_max_clusters_variant<false, kActNone>();
+    return sparse ? pair_max_clusters_variant<true, kActGeluTanh, false>()
+                  : pair_max_clusters_variant<false, kActGeluTanh, false>();
+  return sparse ? pair_max_clusters_variant<true, kActNone, false>() : pair_max_clusters_variant<false, kActNone, false>();
 }
 
 cudaError_t launch_gemm_pair(const GemmLaunch& p, cudaStream_t stream) {
+  if (p.fused)
+    return p.act == kActGeluTanh ? launch_pair_variant<true, kActGeluTanh, true>(p, stream)
+                                 : launch_pair_variant<true, kActNone, true>(p, stream);
   if (p.act == kActGeluTanh)
-    return p.sparse ? launch_pair_variant<true, kActGeluTanh>(p, stream)
-                    : launch_pair_variant<false, kActGeluTanh>(p, stream);
-  return p.sparse ? launch_pair_variant<true, kActNone>(p, stream)
-                  : launch_pair_variant<false, kActNone>(p, stream);
+    return p.sparse ? launch_pair_variant<true, kActGeluTanh, false>(p, stream)
+                    : launch_pair_variant<false, kActGeluTanh, false>(p, stream);
+  return p.sparse ? launch_pair_variant<true, kActNone, false>(p, stream)
+                  : launch_pair_variant<false, kActNone, false>(p, stream);
 }
 
 }  // namespace lynx

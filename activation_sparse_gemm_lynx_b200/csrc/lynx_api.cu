@@ -249,7 +249,7 @@ lynx_status run_sparsify(DeviceState* ds, const void* X, const void* A, int64_t 
     if (!encode_bf16_2d(&p.tm_a, A, K, r, K * 2, 64, static_cast<uint32_t>(r), CU_TENSOR_MAP_SWIZZLE_128B))
       return LYNX_ERR_CUDA;
   }
-  if (mode & kModeSelect) {
+  if ((mode & kModeSelect) && !(mode & kModeNoOut)) {
     // kept values leave through TMA stores of 128 x 32 tiles
     if (!encode_bf16_2d(&p.tm_vals, vals, K / 2, M, K, 32, 128, CU_TENSOR_MAP_SWIZZLE_64B))
       return LYNX_ERR_CUDA;
@@ -283,16 +283,24 @@ bool use_pair_kernel(int64_t M, int64_t N, int64_t K) {
   return M > 128 && N >= 256 && K % 128 == 0;
 }
 
+// fused_x: a_src is the dense X and the pair kernel compresses it itself (the
+// shape must take the pair kernel; no metadata is read)
 lynx_status run_gemm(DeviceState* ds, const void* a_src, bool sparse, const void* meta,
                      const float* row_scale, const void* T, const void* W, const void* bias,
                      const void* B, int64_t M, int64_t N, int64_t K, int64_t r, void* Y,
-                     cudaStream_t stream, const FusedFinalize* fin = nullptr, int act = kActNone) {
+                     cudaStream_t stream, const FusedFinalize* fin = nullptr, int act = kActNone,
+                     bool fused_x = false) {
   GemmLaunch p;
   std::memset(&p, 0, sizeof(p));
   const bool pair = use_pair_kernel(M, N, K);
+  if (fused_x && !pair) return LYNX_ERR_UNSUPPORTED_SHAPE;
   const int bn = pair ? 256 : gemm_bn(N);
   const uint32_t b_rows = pair ? 128u : static_cast<uint32_t>(bn);  // W rows one CTA loads
-  if (sparse) {
+  if (fused_x) {
+    // the dense X in 128 x 64 boxes, as on the dense path
+    if (!encode_bf16_2d(&p.tm_a, a_src, K, M, K * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B))
+      return LYNX_ERR_CUDA;
+  } else if (sparse) {
     // pair kernel: 128-byte rows of 64 kept values; single-CTA kernel: 64-byte rows
     if (!encode_bf16_2d(&p.tm_a, a_src, K / 2, M, K, pair ? 64 : 32, 128,
                         pair ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B))
@@ -332,13 +340,14 @@ lynx_status run_gemm(DeviceState* ds, const void* a_src, bool sparse, const void
   p.bn = bn;
   p.stall_test = g_stall.load();
   p.act = act;
+  p.fused = fused_x ? 1 : 0;
   p.status = stream_status(ds, stream);
   if (pair) {
     const int64_t ntm2 = (M + 255) / 256;
     const int64_t tiles = ntm2 * ((N + 255) / 256);
     // one CTA pair per TPC, no more pairs than the device can hold at once
     int64_t pairs = ds->sms / 2;
-    const int fit = gemm_pair_max_clusters(sparse, act);
+    const int fit = gemm_pair_max_clusters(sparse, act, fused_x);
     if (fit > 0 && fit < pairs) pairs = fit;
     p.grid = static_cast<int>(2 * (tiles < pairs ? tiles : pairs));
     // raster group: as many 256-row pair-rows of A as fit in ~40 MB of L2, so
@@ -561,6 +570,49 @@ int lynx_linear_act(const void* X, const void* W, const void* bias, const void* 
     if (cudaEventRecord(static_cast<cudaEvent_t>(ev), s) != cudaSuccess) return LYNX_ERR_CUDA;
   return run_gemm(ds, X, false, nullptr, nullptr, t_buf, W, bias, B, M, N, K, r, Y, s,
                   fused ? &fin : nullptr, act);
+}
+
+int lynx_linear_fused(const void* X, const void* W, const void* bias, const void* A, const void* B,
+                      int64_t M, int64_t N, int64_t K, int64_t r, int act, void* Y, void* workspace,
+                      size_t workspace_bytes, void* stream) {
+  if (X == nullptr || W == nullptr || Y == nullptr) return LYNX_ERR_INVALID_ARG;
+  if (act != LYNX_ACT_NONE && act != LYNX_ACT_GELU_TANH) return LYNX_ERR_INVALID_ARG;
+  lynx_status st = check_lora(A, B, r);
+  if (st != LYNX_OK) return st;
+  st = check_shape(M, N, K);
+  if (st != LYNX_OK) return st;
+  // shapes the CTA-pair kernel does not take run the two-pass layer
+  if (!use_pair_kernel(M, N, K))
+    return lynx_linear_act(X, W, bias, A, B, M, N, K, r, 0, act, Y, workspace, workspace_bytes, stream);
+  if (!aligned16(X) || !aligned16(W) || !aligned16(Y) || (bias && !aligned16(bias)) ||
+      (A && !aligned16(A)) || (B && !aligned16(B)) || (workspace && !aligned16(workspace)))
+    return LYNX_ERR_MISALIGNED;
+  const WorkspaceLayout wl = workspace_layout(M, K, r);
+  if (workspace == nullptr) return LYNX_ERR_INVALID_ARG;
+  if (workspace_bytes < wl.total) return LYNX_ERR_WORKSPACE_TOO_SMALL;
+  DeviceState* ds = device_state();
+  if (ds == nullptr) return LYNX_ERR_CUDA;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const bool lora = A != nullptr;
+  void* t_buf = lora ? ws + wl.t : nullptr;
+  FusedFinalize fin;
+  fin.mode = 1;
+  fin.split = choose_sparsify_split(M, K, ds->sms);
+  fin.lpart = reinterpret_cast<const float2*>(ws + wl.lpart);
+  fin.tpart = reinterpret_cast<const float*>(ws + wl.tpart);
+  fin.scale = reinterpret_cast<float*>(ws + wl.scale);
+  fin.t = t_buf;
+  fin.flags = reinterpret_cast<uint32_t*>(ws + wl.flags);
+  // the slim pass: the row sums (the selection decides the kept sum) and
+  // T = X A^T, no values or metadata
+  st = run_sparsify(ds, X, A, M, K, r, nullptr, nullptr, reinterpret_cast<float*>(ws + wl.scale), t_buf,
+                    reinterpret_cast<float2*>(ws + wl.lpart), reinterpret_cast<float*>(ws + wl.tpart),
+                    kModeSelect | kModeNoOut | (lora ? kModeLora : 0), s, &fin);
+  if (st != LYNX_OK) return st;
+  if (void* ev = g_split_event.load())
+    if (cudaEventRecord(static_cast<cudaEvent_t>(ev), s) != cudaSuccess) return LYNX_ERR_CUDA;
+  return run_gemm(ds, X, true, nullptr, nullptr, t_buf, W, bias, B, M, N, K, r, Y, s, &fin, act, true);
 }
 
 size_t lynx_linear_host_workspace_bytes(int64_t M, int64_t N, int64_t K, int64_t r) {

@@ -23,8 +23,10 @@ constexpr int kMetaBlockBytes = 2048;  // 128 TMEM lanes x 16 bytes
 
 // kModeSelect: S(X) (kept values + metadata + s); kModeLora: T = X A^T;
 // kModeScaled: values leave compensated (standalone S(X)), otherwise they
-// leave as kept and s is applied by the GEMM (T is then written as T / s).
-enum SparsifyMode : int { kModeSelect = 1, kModeLora = 2, kModeScaled = 4 };
+// leave as kept and s is applied by the GEMM (T is then written as T / s);
+// kModeNoOut (with kModeSelect): the selection only feeds the row sums, no
+// values or metadata are written (the fused GEMM selects again from X).
+enum SparsifyMode : int { kModeSelect = 1, kModeLora = 2, kModeScaled = 4, kModeNoOut = 8 };
 
 // Activation the GEMM epilogue applies to each finished output value (the
 // LYNX_ACT_* values of the public header).
@@ -104,6 +106,7 @@ struct GemmLaunch {
   int group_m;          // tile rows (of 128 or of 256 for CTA pairs) per raster group
   int stall_test;
   int act;              // EpilogueAct
+  int fused;            // pair kernel: A is the dense X, compressed in the kernel (tm_a maps X)
   uint32_t* status;
   // Combining the sparsify pass's K-range partials inside the pair GEMM (instead
   // of finalize_kernel): fin_mode 1 = s (and, with LoRA, bf16(T / s)), 2 =
@@ -126,7 +129,7 @@ cudaError_t launch_gemm(const GemmLaunch& p, cudaStream_t stream);       // 128 
 cudaError_t launch_gemm_pair(const GemmLaunch& p, cudaStream_t stream);  // 256 x 256 tiles, CTA pairs
 // CTA pairs of the pair GEMM (this variant) that the current device can hold at
 // once; 0 if the query failed.  Computed once per device and variant.
-int gemm_pair_max_clusters(bool sparse, int act);
+int gemm_pair_max_clusters(bool sparse, int act, bool fused = false);
 
 // Per-device one-time set-up of a kernel's dynamic shared-memory limit:
 // `configure` runs once for each device (thread-safe); its result is kept.

@@ -46,6 +46,7 @@
 
 #include "lynx_internal.h"
 #include "lynx_ptx.cuh"
+#include "lynx_select.cuh"
 
 namespace lynx {
 
@@ -101,53 +102,6 @@ __host__ __device__ inline uint32_t lora_tmem_cols(int r) {
   return c;
 }
 
-// acc_lo += low bf16 of w, acc_hi += high bf16 of w, in fp32 (one rounding
-// each; the bf16 operand is exact in fp32)
-__device__ __forceinline__ void add_bf16_pair(float& acc_lo, float& acc_hi, uint32_t w) {
-  asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %2;\n\t"
-      "add.rn.f32.bf16 %0, lo, %0;\n\tadd.rn.f32.bf16 %1, hi, %1;\n\t}"
-      : "+f"(acc_lo), "+f"(acc_hi)
-      : "r"(w));
-}
-
-// per 16-bit lane: 0xFFFF if a >= b, else 0 (bf16 compare; for the
-// non-negative finite magnitudes used here the order of the bit patterns)
-__device__ __forceinline__ uint32_t ge_bf16x2(uint32_t a, uint32_t b) {
-  uint32_t r;
-  asm("set.ge.u32.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
-  return r;
-}
-
-// The selection of a group of 4 is decided by the six comparisons
-// "x_i beats x_j" (i < j): |x_i| >= |x_j|, so a tie goes to the lower index.
-// They come out of three bf16x2 compares as a 6-bit code,
-//   bit 0: |x0| >= |x2|   bit 1: |x0| >= |x3|   bit 2: |x0| >= |x1|
-//   bit 3: |x1| >= |x3|   bit 4: |x1| >= |x2|   bit 5: |x2| >= |x3|,
-// and a 64-entry table gives, per code, the byte selector that packs the two
-// kept values (lower position in the low half) and the nibble lo | hi << 2.
-// Value i is kept when fewer than two values beat it; a code that no order of
-// four magnitudes produces maps to the two least beaten values.
-__device__ __forceinline__ uint32_t selection_table_entry(uint32_t code) {
-  const int p02 = code & 1, p03 = (code >> 1) & 1, p01 = (code >> 2) & 1;
-  const int p13 = (code >> 3) & 1, p12 = (code >> 4) & 1, p23 = (code >> 5) & 1;
-  const int beaten[4] = {(1 - p01) + (1 - p02) + (1 - p03), p01 + (1 - p12) + (1 - p13),
-                         p02 + p12 + (1 - p23), p03 + p13 + p23};
-  int lo = -1, hi = -1;
-  for (int limit = 0; limit <= 3 && hi < 0; ++limit)  // the least beaten first, lower index first
-    for (int i = 0; i < 4 && hi < 0; ++i)
-      if (beaten[i] == limit && i != lo) {
-        if (lo < 0) lo = i;
-        else hi = i;
-      }
-  if (hi < lo) {
-    const int t = lo;
-    lo = hi;
-    hi = t;
-  }
-  const uint32_t sel = (2u * lo) | ((2u * lo + 1u) << 4) | ((2u * hi) << 8) | ((2u * hi + 1u) << 12);
-  return sel | ((static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 2)) << 16);
-}
-
 // Top-2 of the 4 bf16 values in (w0 = x1:x0, w1 = x3:x2) by magnitude, ties to
 // the lower index, together with the group's terms of the row's two L1 sums:
 // |x0|, |x2| to la_even and |x1|, |x3| to la_odd, the kept magnitudes to lk_lo
@@ -160,12 +114,7 @@ __device__ __forceinline__ uint32_t select_group(uint32_t w0, uint32_t w1, const
   const uint32_t a1 = w1 & 0x7FFF7FFFu;  // |x3| : |x2|
   add_bf16_pair(la_even, la_odd, a0);
   add_bf16_pair(la_even, la_odd, a1);
-  const uint32_t c1 = ge_bf16x2(a0, a1);                                // x0>=x2 | x1>=x3
-  const uint32_t c2 = ge_bf16x2(a0, __byte_perm(a1, 0, 0x1032));        // x0>=x3 | x1>=x2
-  const uint32_t c3 = ge_bf16x2(__byte_perm(a0, a1, 0x5410), __byte_perm(a0, a1, 0x7632));  // x0>=x1 | x2>=x3
-  uint32_t code = (c1 & 0x00010001u) | (c2 & 0x00020002u) | (c3 & 0x00040004u);
-  code = (code | (code >> 13)) & 0x3Fu;
-  const uint32_t ent = table[code];
+  const uint32_t ent = table[selection_code(a0, a1)];
   kept = __byte_perm(w0, w1, ent);
   add_bf16_pair(lk_lo, lk_hi, __byte_perm(a0, a1, ent));
   return ent >> 16;
@@ -188,6 +137,7 @@ sparsify_kernel(const __grid_constant__ SparsifyLaunch p) {
   extern __shared__ uint8_t smem_raw[];
   const bool do_sel = (p.mode & kModeSelect) != 0;
   const bool do_lora = (p.mode & kModeLora) != 0;
+  const bool write_out = do_sel && (p.mode & kModeNoOut) == 0;  // values and metadata leave
   const SparsifyLayout lay = sparsify_layout(do_lora, p.r);
   uint8_t* base = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -264,7 +214,7 @@ sparsify_kernel(const __grid_constant__ SparsifyLaunch p) {
     // hands back the buffer of the previous box's store, which has read it by
     // then (vfree).  The last box's buffer is not needed again.
     if (lane == 0) {
-      if (do_sel) tma_prefetch_desc(&p.tm_vals);
+      if (write_out) tma_prefetch_desc(&p.tm_vals);
       const uint32_t tx = kXTileBytes + lay.a_tile;
       const bool store_rows = mb * 128 < p.M;  // a padding row block has metadata only
       bool ok = !p.stall_test;
@@ -280,7 +230,9 @@ sparsify_kernel(const __grid_constant__ SparsifyLaunch p) {
               set_abort(sm, p.status, kDevTimeoutEmpty);
               break;
             }
-            if (store_rows) {
+            if (!write_out) {
+              // nothing staged: the stage is free once the row threads are done
+            } else if (store_rows) {
               tma_store_2d(&p.tm_vals, vstage + (prev & 1) * kStoreTileBytes,
                            static_cast<int32_t>((kcol0 + 64 * prev) / 2),
                            static_cast<int32_t>(mb * 128));
@@ -404,20 +356,22 @@ sparsify_kernel(const __grid_constant__ SparsifyLaunch p) {
       const uint32_t n5 = select_group(v2.z, v2.w, tab, kw[5], la0, la1, lk0, lk1);
       const uint32_t n6 = select_group(v3.x, v3.y, tab, kw[6], la0, la1, lk0, lk1);
       const uint32_t n7 = select_group(v3.z, v3.w, tab, kw[7], la0, la1, lk0, lk1);
-      meta_ptr[0] = static_cast<uint16_t>(n0 + n1 * 16u + n2 * 256u + n3 * 4096u);
-      meta_ptr[64] = static_cast<uint16_t>(n4 + n5 * 16u + n6 * 256u + n7 * 4096u);
-      meta_ptr += meta_hi_half ? 1020 : 4;
-      meta_hi_half ^= 1u;
-      // the store of box b - 2 has read this staging buffer
-      if (!mbar_wait(&sm.vfree[b & 1], static_cast<uint32_t>((b >> 1) & 1) ^ 1u)) {
-        set_abort(sm, p.status, kDevTimeoutEmpty);
-        ok = false;
+      if (write_out) {
+        meta_ptr[0] = static_cast<uint16_t>(n0 + n1 * 16u + n2 * 256u + n3 * 4096u);
+        meta_ptr[64] = static_cast<uint16_t>(n4 + n5 * 16u + n6 * 256u + n7 * 4096u);
+        meta_ptr += meta_hi_half ? 1020 : 4;
+        meta_hi_half ^= 1u;
+        // the store of box b - 2 has read this staging buffer
+        if (!mbar_wait(&sm.vfree[b & 1], static_cast<uint32_t>((b >> 1) & 1) ^ 1u)) {
+          set_abort(sm, p.status, kDevTimeoutEmpty);
+          ok = false;
+        }
+        if (!__all_sync(0xffffffffu, ok)) break;
+        uint8_t* const vbuf = vstage + (b & 1) * kStoreTileBytes;
+        *reinterpret_cast<uint4*>(vbuf + vst_off0) = make_uint4(kw[0], kw[1], kw[2], kw[3]);
+        *reinterpret_cast<uint4*>(vbuf + vst_off1) = make_uint4(kw[4], kw[5], kw[6], kw[7]);
+        fence_proxy_async_smem();
       }
-      if (!__all_sync(0xffffffffu, ok)) break;
-      uint8_t* const vbuf = vstage + (b & 1) * kStoreTileBytes;
-      *reinterpret_cast<uint4*>(vbuf + vst_off0) = make_uint4(kw[0], kw[1], kw[2], kw[3]);
-      *reinterpret_cast<uint4*>(vbuf + vst_off1) = make_uint4(kw[4], kw[5], kw[6], kw[7]);
-      fence_proxy_async_smem();
       // release the stage only after everything derived from it has been
       // produced: an arrive does not wait for this warp's loads in flight
       __syncwarp();

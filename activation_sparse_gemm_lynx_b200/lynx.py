@@ -62,6 +62,7 @@ def library():
             "lynx_linear": ([p, p, p, p, p, i64, i64, i64, i64, i32, p, p, sz, p], i32),
             "lynx_linear_act": ([p, p, p, p, p, i64, i64, i64, i64, i32, i32, p, p, sz, p], i32),
             "lynx_linear_dense": ([p, p, p, p, p, i64, i64, i64, i64, p, p, sz, p], i32),
+            "lynx_linear_fused": ([p, p, p, p, p, i64, i64, i64, i64, i32, p, p, sz, p], i32),
             "lynx_linear_host_workspace_bytes": ([i64, i64, i64, i64], sz),
             "lynx_linear_host": ([p, p, p, p, p, i64, i64, i64, i64, i32, p, p, sz, p], i32),
             "lynx_linear_host_act": ([p, p, p, p, p, i64, i64, i64, i64, i32, i32, p, p, sz, p], i32),
@@ -262,6 +263,18 @@ def lynx_linear_act(X, W, bias=None, A=None, B=None, skip_sparsify=False, act=LY
                                    1 if skip_sparsify else 0, int(act), _ptr(Y), _ptr(workspace),
                                    workspace.numel(), _stream(stream))
     _check(st, "lynx_linear_act")
+    return Y
+
+
+def lynx_linear_fused(X, W, bias=None, A=None, B=None, act=LYNX_ACT_NONE, Y=None, workspace=None,
+                      stream=None):
+    """The fully fused variant: the 2:4 selection and compression inside the
+    GEMM, after a slim pass for s and T (see include/lynx.h).  Returns Y."""
+    M, N, K, r, Y, workspace = _linear_buffers(X, W, bias, A, B, Y, workspace)
+    st = library().lynx_linear_fused(_ptr(X), _ptr(W), _ptr(bias), _ptr(A), _ptr(B), M, N, K, r,
+                                     int(act), _ptr(Y), _ptr(workspace), workspace.numel(),
+                                     _stream(stream))
+    _check(st, "lynx_linear_fused")
     return Y
 
 

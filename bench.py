@@ -353,6 +353,9 @@ class LayerTimer:
         if self.act != self.lynx.LYNX_ACT_NONE:
             self.torch.nn.functional.gelu(self.Yd, approximate="tanh")
 
+    def step_fused(self):
+        self.lynx.lynx_linear_fused(self.X, self.W, self.bias, self.A, self.B, Y=self.Y, workspace=self.ws)
+
     def step_unfused_act(self):
         # the plain layer, then the activation as a pass of its own over Y
         self.lynx.lynx_linear(self.X, self.W, self.bias, self.A, self.B, Y=self.Y, workspace=self.ws)
@@ -425,7 +428,7 @@ def stored_gemm_traffic(workload):
     return rec["bytes"], f"ncu capture of {rec['captured']} (sources {rec['src']})"
 
 
-def layer_summary(lt, ms_linear, parts, dense_ms, peaks, clock_info=None):
+def layer_summary(lt, ms_linear, parts, dense_ms, peaks, clock_info=None, fused_ms=None):
     M, N, K, r = lt.shape.M, lt.shape.N, lt.shape.K, lt.shape.r
     flops = 2.0 * M * N * K
     sparse_peak = 2.0 * peaks["bf16_tflops"]
@@ -440,6 +443,10 @@ def layer_summary(lt, ms_linear, parts, dense_ms, peaks, clock_info=None):
         "ms": {"sparsify_kernel": parts["sparsify_kernel"], "gemm_kernel": parts["gemm_kernel"],
                "dense_torch_matmul": dense_ms},
     }
+    if fused_ms is not None:
+        # the fully fused variant (selection inside the GEMM), for comparison
+        out["fused_variant"] = {"ms_per_step": fused_ms, "value": flops / (fused_ms * 1e-3) / 1e12,
+                                "vs_two_pass": ms_linear / fused_ms}
     if clock_info is not None:
         out["clocks"] = clock_info
     return out
@@ -623,9 +630,14 @@ def run_lynx(args):
     # way (fewer steps); the headline stays the selected workload
     if not args.no_per_config and act == lynx.LYNX_ACT_NONE:
         per = {}
+        def fused_time(t):
+            for _ in range(3):
+                t.step_fused()
+            return max_over_ranks(statistics.mean(t.timed(t.step_fused, ncmp)), world)
+
         for name in ("attn_out", "mlp_up", "mlp_down"):
             if name == args.workload:
-                per[name] = layer_summary(lt, ms_step, parts, dense_ms, peaks, clock_info)
+                per[name] = layer_summary(lt, ms_step, parts, dense_ms, peaks, clock_info, fused_time(lt))
                 continue
             other = LayerTimer(name, rank, "none", flush)
             for _ in range(max(3, args.warmup)):
@@ -641,7 +653,7 @@ def run_lynx(args):
             for _ in range(3):
                 other.step_dense_torch()
             o_dense = max_over_ranks(statistics.mean(other.timed(other.step_dense_torch, ncmp)), world)
-            per[name] = layer_summary(other, o_ms, o_parts, o_dense, peaks, o_clock)
+            per[name] = layer_summary(other, o_ms, o_parts, o_dense, peaks, o_clock, fused_time(other))
             per[name]["steps"] = ncmp
             del other
         st, code = lynx.lynx_check_error()

@@ -209,6 +209,26 @@ LYNX_API int lynx_linear_act(const void* X, const void* W, const void* bias, con
                              int skip_sparsify, int act, void* Y, void* workspace,
                              size_t workspace_bytes, void* stream);
 
+/* ---- the fully fused variant ------------------------------------------- */
+
+/* Y = act(S(X) W^T + bias + (X A^T) B^T) like lynx_linear_act, with the 2:4
+ * selection and compression inside the GEMM (qingkeai.online article, section
+ * 04: selection, compression, the sparse operand layout, the sparse GEMM and the
+ * LoRA residual fused, no compressed activations written back).  A slim first
+ * pass reads X for the two row sums (s) and T = X A^T only; the GEMM then loads
+ * the dense X tiles itself, selects and compresses them in shared memory into
+ * the tcgen05.mma.sp operand (values and metadata) and multiplies.  The
+ * selection is redone for every output tile of 256 columns, so on B200 this
+ * variant is slower than lynx_linear whenever N is much more than 256 (the
+ * selection work grows with N / 256); lynx_linear is the default path.
+ * Results equal lynx_linear's within the same tolerance (the same s, the same
+ * kept values).  Arguments, workspace and errors as lynx_linear_act without
+ * skip_sparsify; shapes the CTA-pair GEMM does not take (M <= 128, N < 256,
+ * K % 128 != 0) run lynx_linear_act. */
+LYNX_API int lynx_linear_fused(const void* X, const void* W, const void* bias, const void* A,
+                               const void* B, int64_t M, int64_t N, int64_t K, int64_t r, int act,
+                               void* Y, void* workspace, size_t workspace_bytes, void* stream);
+
 /* ---- the layer on host-memory activations ------------------------------ */
 
 /* Bytes of the device workspace lynx_linear_host needs: device copies of X and
