@@ -20,7 +20,9 @@ from .lynx import (  # noqa: F401
     lynx_debug_set_stall,
     lynx_linear,
     lynx_linear_act,
+    lynx_linear_begin,
     lynx_linear_dense,
+    lynx_linear_finish,
     lynx_linear_fused,
     lynx_linear_host,
     lynx_linear_host_act,

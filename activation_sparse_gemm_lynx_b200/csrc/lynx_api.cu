@@ -505,9 +505,18 @@ int lynx_linear(const void* X, const void* W, const void* bias, const void* A, c
                          workspace_bytes, stream);
 }
 
-int lynx_linear_act(const void* X, const void* W, const void* bias, const void* A, const void* B,
-                    int64_t M, int64_t N, int64_t K, int64_t r, int skip_sparsify, int act, void* Y,
-                    void* workspace, size_t workspace_bytes, void* stream) {
+}  // extern "C"
+
+namespace {
+
+// The layer's two halves on `stream`: begin = the sparsify pass (or, on the
+// dense path with LoRA, the LoRA-down pass) into the workspace; finish = the
+// GEMM from it.  reset_flags: finish alone on a workspace an earlier call
+// filled (profiling), which first clears the combining step's state words.
+lynx_status linear_enqueue(const void* X, const void* W, const void* bias, const void* A, const void* B,
+                           int64_t M, int64_t N, int64_t K, int64_t r, int skip_sparsify, int act, void* Y,
+                           void* workspace, size_t workspace_bytes, cudaStream_t s, bool do_begin,
+                           bool do_finish, bool reset_flags) {
   if (X == nullptr || W == nullptr || Y == nullptr) return LYNX_ERR_INVALID_ARG;
   if (act != LYNX_ACT_NONE && act != LYNX_ACT_GELU_TANH) return LYNX_ERR_INVALID_ARG;
   lynx_status st = check_lora(A, B, r);
@@ -524,7 +533,6 @@ int lynx_linear_act(const void* X, const void* W, const void* bias, const void* 
     return workspace == nullptr ? LYNX_ERR_INVALID_ARG : LYNX_ERR_WORKSPACE_TOO_SMALL;
   DeviceState* ds = device_state();
   if (ds == nullptr) return LYNX_ERR_CUDA;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   void* t_buf = lora ? ws + wl.t : nullptr;
   // with the CTA-pair GEMM, the GEMM itself combines the pass's K-range partials
@@ -539,37 +547,53 @@ int lynx_linear_act(const void* X, const void* W, const void* bias, const void* 
     fin.t = t_buf;
     fin.flags = reinterpret_cast<uint32_t*>(ws + wl.flags);
   }
-  const int part = g_profile_part.load();
-  if (!skip_sparsify) {
-    if (part != 2) {
-      st = run_sparsify(ds, X, A, M, K, r, ws + wl.vals, ws + wl.meta,
-                        reinterpret_cast<float*>(ws + wl.scale), t_buf,
-                        reinterpret_cast<float2*>(ws + wl.lpart), reinterpret_cast<float*>(ws + wl.tpart),
+  if (do_begin) {
+    if (!skip_sparsify) {
+      st = run_sparsify(ds, X, A, M, K, r, ws + wl.vals, ws + wl.meta, reinterpret_cast<float*>(ws + wl.scale),
+                        t_buf, reinterpret_cast<float2*>(ws + wl.lpart), reinterpret_cast<float*>(ws + wl.tpart),
                         kModeSelect | (lora ? kModeLora : 0), s, fused ? &fin : nullptr);
-      if (st != LYNX_OK || part == 1) return st;
-    } else if (fused && cudaMemsetAsync(fin.flags, 0, fin_slices(M) * 4, s) != cudaSuccess) {
-      return LYNX_ERR_CUDA;
-    }
-    if (void* ev = g_split_event.load())
-      if (cudaEventRecord(static_cast<cudaEvent_t>(ev), s) != cudaSuccess) return LYNX_ERR_CUDA;
-    return run_gemm(ds, ws + wl.vals, true, ws + wl.meta, reinterpret_cast<const float*>(ws + wl.scale),
-                    t_buf, W, bias, B, M, N, K, r, Y, s, fused ? &fin : nullptr, act);
-  }
-  if (lora) {
-    if (part != 2) {
+    } else if (lora) {
       st = run_sparsify(ds, X, A, M, K, r, nullptr, nullptr, nullptr, t_buf, nullptr,
                         reinterpret_cast<float*>(ws + wl.tpart), kModeLora, s, fused ? &fin : nullptr);
-      if (st != LYNX_OK || part == 1) return st;
-    } else if (fused && cudaMemsetAsync(fin.flags, 0, fin_slices(M) * 4, s) != cudaSuccess) {
-      return LYNX_ERR_CUDA;
     }
-  } else if (part == 1) {
-    return LYNX_OK;
+    if (st != LYNX_OK) return st;
   }
+  if (!do_finish) return LYNX_OK;
+  if (reset_flags && fused && cudaMemsetAsync(fin.flags, 0, fin_slices(M) * 4, s) != cudaSuccess)
+    return LYNX_ERR_CUDA;
   if (void* ev = g_split_event.load())
     if (cudaEventRecord(static_cast<cudaEvent_t>(ev), s) != cudaSuccess) return LYNX_ERR_CUDA;
+  if (!skip_sparsify)
+    return run_gemm(ds, ws + wl.vals, true, ws + wl.meta, reinterpret_cast<const float*>(ws + wl.scale),
+                    t_buf, W, bias, B, M, N, K, r, Y, s, fused ? &fin : nullptr, act);
   return run_gemm(ds, X, false, nullptr, nullptr, t_buf, W, bias, B, M, N, K, r, Y, s,
                   fused ? &fin : nullptr, act);
+}
+
+}  // namespace
+
+extern "C" {
+
+int lynx_linear_act(const void* X, const void* W, const void* bias, const void* A, const void* B,
+                    int64_t M, int64_t N, int64_t K, int64_t r, int skip_sparsify, int act, void* Y,
+                    void* workspace, size_t workspace_bytes, void* stream) {
+  const int part = g_profile_part.load();
+  return linear_enqueue(X, W, bias, A, B, M, N, K, r, skip_sparsify, act, Y, workspace, workspace_bytes,
+                        static_cast<cudaStream_t>(stream), part != 2, part != 1, part == 2);
+}
+
+int lynx_linear_begin(const void* X, const void* W, const void* bias, const void* A, const void* B,
+                      int64_t M, int64_t N, int64_t K, int64_t r, int skip_sparsify, int act, void* Y,
+                      void* workspace, size_t workspace_bytes, void* stream) {
+  return linear_enqueue(X, W, bias, A, B, M, N, K, r, skip_sparsify, act, Y, workspace, workspace_bytes,
+                        static_cast<cudaStream_t>(stream), true, false, false);
+}
+
+int lynx_linear_finish(const void* X, const void* W, const void* bias, const void* A, const void* B,
+                       int64_t M, int64_t N, int64_t K, int64_t r, int skip_sparsify, int act, void* Y,
+                       void* workspace, size_t workspace_bytes, void* stream) {
+  return linear_enqueue(X, W, bias, A, B, M, N, K, r, skip_sparsify, act, Y, workspace, workspace_bytes,
+                        static_cast<cudaStream_t>(stream), false, true, false);
 }
 
 int lynx_linear_fused(const void* X, const void* W, const void* bias, const void* A, const void* B,

@@ -61,6 +61,8 @@ def library():
             "lynx_sparsify_noalloc_max_rows": ([], i64),
             "lynx_linear": ([p, p, p, p, p, i64, i64, i64, i64, i32, p, p, sz, p], i32),
             "lynx_linear_act": ([p, p, p, p, p, i64, i64, i64, i64, i32, i32, p, p, sz, p], i32),
+            "lynx_linear_begin": ([p, p, p, p, p, i64, i64, i64, i64, i32, i32, p, p, sz, p], i32),
+            "lynx_linear_finish": ([p, p, p, p, p, i64, i64, i64, i64, i32, i32, p, p, sz, p], i32),
             "lynx_linear_dense": ([p, p, p, p, p, i64, i64, i64, i64, p, p, sz, p], i32),
             "lynx_linear_fused": ([p, p, p, p, p, i64, i64, i64, i64, i32, p, p, sz, p], i32),
             "lynx_linear_host_workspace_bytes": ([i64, i64, i64, i64], sz),
@@ -264,6 +266,29 @@ def lynx_linear_act(X, W, bias=None, A=None, B=None, skip_sparsify=False, act=LY
                                    workspace.numel(), _stream(stream))
     _check(st, "lynx_linear_act")
     return Y
+
+
+def _linear_half(name, X, W, bias, A, B, skip_sparsify, act, Y, workspace, stream):
+    M, N, K, r, Y, workspace = _linear_buffers(X, W, bias, A, B, Y, workspace)
+    st = getattr(library(), name)(_ptr(X), _ptr(W), _ptr(bias), _ptr(A), _ptr(B), M, N, K, r,
+                                  1 if skip_sparsify else 0, int(act), _ptr(Y), _ptr(workspace),
+                                  workspace.numel(), _stream(stream))
+    _check(st, name)
+    return Y
+
+
+def lynx_linear_begin(X, W, bias=None, A=None, B=None, skip_sparsify=False, act=LYNX_ACT_NONE, Y=None,
+                      workspace=None, stream=None):
+    """First half of lynx_linear_act: the sparsify (or LoRA-down) pass into
+    `workspace` (see include/lynx.h).  Returns Y (not yet written)."""
+    return _linear_half("lynx_linear_begin", X, W, bias, A, B, skip_sparsify, act, Y, workspace, stream)
+
+
+def lynx_linear_finish(X, W, bias=None, A=None, B=None, skip_sparsify=False, act=LYNX_ACT_NONE, Y=None,
+                       workspace=None, stream=None):
+    """Second half of lynx_linear_act: the GEMM from the workspace a completed
+    lynx_linear_begin filled.  Returns Y."""
+    return _linear_half("lynx_linear_finish", X, W, bias, A, B, skip_sparsify, act, Y, workspace, stream)
 
 
 def lynx_linear_fused(X, W, bias=None, A=None, B=None, act=LYNX_ACT_NONE, Y=None, workspace=None,

@@ -82,6 +82,8 @@ def parse_args(argv=None):
     ap.add_argument("--gather-y", action="store_true",
                     help="with --gpus N > 1: also time the layer followed by an all-gather of Y "
                          "(every rank ends with all N x M rows), reported as y_gather")
+    ap.add_argument("--sweep-schedule", choices=["serial", "overlap", "overlap_chunks2"], default="serial",
+                    help="--workload sweep: the schedule the headline times (all three are reported)")
     ap.add_argument("--only-linear", action="store_true",
                     help="time the layer only (no comparisons, e2e or CPU baseline); "
                          "the short launch sequence used for ncu captures")
@@ -673,11 +675,6 @@ def run_lynx(args):
     return 0
 
 
-def _mkn(t):
-    M, K, N = t["shape"]
-    return M, N, K
-
-
 def run_sweep(args):
     """The DiT block sweep: 8 blocks x {qkv, out, up, down} linears at M = 8192,
     2 blocks left dense (skip_sparsify), fresh seeded inputs per linear, all 32
@@ -732,7 +729,15 @@ def run_sweep(args):
     if st != lynx.LYNX_OK:
         raise RuntimeError(f"device status after the first pass: {st} code {code:#x}")
     eager_before = timed(sweep.run, 5)
-    sweep.capture()
+    # the other schedules, each run once eagerly before its capture
+    schedules = {"serial": (False, 1), "overlap": (True, 1), "overlap_chunks2": (True, 2)}
+    graphs = {}
+    for name, (overlapped, chunks) in schedules.items():
+        if overlapped:
+            sweep.run_overlapped(chunks)
+            torch.cuda.synchronize()
+        graphs[name] = sweep.capture(overlapped, chunks)
+    sweep.graph = graphs[args.sweep_schedule]
     for _ in range(args.warmup):
         sweep.replay()
     clocks = ClockSampler(local_rank)
@@ -746,6 +751,17 @@ def run_sweep(args):
     if st != lynx.LYNX_OK:
         raise RuntimeError(f"device status after timing: {st} code {code:#x}")
     ms_step = max_over_ranks(sum(tot), world) / args.steps
+    schedule_ms = {}
+    for name, g in graphs.items():
+        for _ in range(3):
+            g.replay()
+        schedule_ms[name] = max_over_ranks(statistics.mean(timed(g.replay, max(3, min(args.steps, 20)))),
+                                           world)
+    st, code = lynx.lynx_check_error()
+    if st == lynx.LYNX_OK and sweep._overlap:
+        st, code = lynx.lynx_check_error(next(iter(sweep._overlap.values()))[0])
+    if st != lynx.LYNX_OK:
+        raise RuntimeError(f"device status after the schedules: {st} code {code:#x}")
     # eager launches (host work in every step) before and after the graph loop
     eager_ms = max_over_ranks(statistics.mean(eager_before + timed(sweep.run, 5)), world)
 
@@ -789,22 +805,28 @@ def run_sweep(args):
             "l2": "flushed before every step (256 MiB write, outside the timed step)",
             "parallelism": f"dp{world} (independent token-row batches per GPU, no collective)",
             "graph": "the 32 lynx_linear calls replayed from one CUDA graph",
+            "schedule": {"serial": "the calls in order on one stream",
+                         "overlap": "each layer's sparsify pass on a side stream, its GEMM on the main "
+                                    "stream, two workspaces in turn",
+                         "overlap_chunks2": "as overlap, each layer in two row blocks"}[args.sweep_schedule],
             **({"act": "GELU(tanh) on the 8 MLP up-projection outputs: in the GEMM epilogue here, "
                        "as a separate torch pass after each matmul in the cuBLAS graph"}
                if gelu_up else {}),
         },
         "speedup_vs_dense_bf16": dense_ms / ms_step,
         "breakdown_ms": {"sweep_graph": ms_step, "sweep_eager": eager_ms,
-                         "dense_torch_matmul_graph": dense_ms},
-        "gpu_launches": args.steps * sum(launches_per_linear(*_mkn(t), skip=t["skip"],
-                                                             lora=t["A"] is not None)
-                                         for t in sweep.layers),
+                         "dense_torch_matmul_graph": dense_ms,
+                         **{f"sweep_graph_{k}": v for k, v in schedule_ms.items()}},
+        "gpu_launches": args.steps * sum(
+            launches_per_linear(r1 - r0, t["shape"][2], t["shape"][1], skip=t["skip"], lora=t["A"] is not None)
+            for (t, r0, r1) in sweep.work_items(schedules[args.sweep_schedule][1])),
         "clocks": clock_info,
     }
     if world > 1:
         import torch.distributed as dist
 
         sweep.graph = None
+        graphs.clear()
         dist.destroy_process_group()
     if rank == 0:
         print(json.dumps(result), flush=True)

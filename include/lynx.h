@@ -177,6 +177,30 @@ LYNX_API int lynx_linear(const void* X, const void* W, const void* bias, const v
                 int64_t M, int64_t N, int64_t K, int64_t r, int skip_sparsify, void* Y,
                 void* workspace, size_t workspace_bytes, void* stream);
 
+/* ---- the layer in two halves ------------------------------------------ */
+
+/* lynx_linear_act split at its one internal hand-off, so that a caller can put
+ * the halves on different streams (for example the next layer's pass beside
+ * this layer's GEMM, each with its own workspace):
+ *   lynx_linear_begin   the sparsify pass (S(X) kept values, metadata, the row
+ *                       sums and T partials) into the workspace; on the dense
+ *                       path (skip_sparsify) the LoRA-down pass, or nothing;
+ *   lynx_linear_finish  the GEMM from that workspace into Y.
+ * Both take lynx_linear_act's arguments and check them the same way.  finish
+ * must run after begin has completed on the same workspace (the same stream in
+ * order, or another stream that waits on an event recorded after begin), with
+ * nothing else writing that workspace in between; then the pair computes
+ * exactly what lynx_linear_act does (the same Y, bit for bit).  begin reads X
+ * and A; finish reads X (dense path only), W, bias, B and the workspace. */
+LYNX_API int lynx_linear_begin(const void* X, const void* W, const void* bias, const void* A,
+                               const void* B, int64_t M, int64_t N, int64_t K, int64_t r,
+                               int skip_sparsify, int act, void* Y, void* workspace,
+                               size_t workspace_bytes, void* stream);
+LYNX_API int lynx_linear_finish(const void* X, const void* W, const void* bias, const void* A,
+                                const void* B, int64_t M, int64_t N, int64_t K, int64_t r,
+                                int skip_sparsify, int act, void* Y, void* workspace,
+                                size_t workspace_bytes, void* stream);
+
 /* ---- an activation applied in the GEMM epilogue ------------------------ */
 
 /* Activations lynx_linear_act applies to the finished output row. */

@@ -138,3 +138,89 @@ def test_sweep_with_gelu_on_up_layers():
                                    np.linalg.norm(helpers.f32(inp["W"]).astype(np.float64), axis=1))
     assert float((np.abs(y - y_ref) / bound).max()) <= 1.0
     assert np.linalg.norm(y - y_ref) <= 1.13 * 5e-3 * np.linalg.norm(y_pre)
+
+
+def dev(bits):
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to("cuda:0")
+
+
+@pytest.mark.parametrize("skip,act,lora", [(False, lynx.LYNX_ACT_NONE, True), (True, lynx.LYNX_ACT_NONE, True),
+                                           (False, lynx.LYNX_ACT_GELU_TANH, True),
+                                           (False, lynx.LYNX_ACT_NONE, False),
+                                           (True, lynx.LYNX_ACT_NONE, False)])
+def test_begin_then_finish_on_two_streams_equals_linear(skip, act, lora):
+    """lynx_linear_begin on one stream and lynx_linear_finish on another (after
+    an event) give the same Y bits as lynx_linear_act, on the mlp_up shape."""
+    torch.cuda.set_device(0)
+    c = workloads.CONFIGS["mlp_up"]
+    inp = workloads.make_config_inputs("mlp_up")
+    X, W, bias, A, B = (dev(inp[k]) for k in ("X", "W", "bias", "A", "B"))
+    if not lora:
+        A = B = None
+    ref = lynx.lynx_linear_act(X, W, bias, A, B, skip_sparsify=skip, act=act)
+    s_begin, s_finish = torch.cuda.Stream(), torch.cuda.Stream()
+    ws = torch.full((lynx.lynx_workspace_bytes(c.M, c.N, c.K, c.r),), 0xA5, dtype=torch.uint8, device="cuda:0")
+    Y = torch.zeros_like(ref)
+    torch.cuda.synchronize()
+    lynx.lynx_linear_begin(X, W, bias, A, B, skip_sparsify=skip, act=act, Y=Y, workspace=ws, stream=s_begin)
+    ev = torch.cuda.Event()
+    ev.record(s_begin)
+    s_finish.wait_event(ev)
+    lynx.lynx_linear_finish(X, W, bias, A, B, skip_sparsify=skip, act=act, Y=Y, workspace=ws, stream=s_finish)
+    torch.cuda.synchronize()
+    for s in (s_begin, s_finish, None):
+        st, code = lynx.lynx_check_error(s)
+        assert st == lynx.LYNX_OK, (st, code)
+    assert torch.equal(Y.view(torch.int16), ref.view(torch.int16))
+
+
+def test_overlapped_schedules_equal_serial_calls(sweep_and_plan):
+    """The overlapped sweep (passes on a side stream, GEMMs on the main one, two
+    workspaces) eagerly and from a graph gives the serial pass's Y bits; with
+    row blocks (384 rows: a 256-row block and a 128-row tail) every block
+    equals a lynx_linear call on the same rows."""
+    sweep, plan, layers = sweep_and_plan
+    sweep.run()
+    torch.cuda.synchronize()
+    serial = [t["Y"].clone() for t in sweep.layers]
+
+    def check(expected, what):
+        torch.cuda.synchronize()
+        st, code = lynx.lynx_check_error()
+        assert st == lynx.LYNX_OK, (what, st, code)
+        for st_side in sweep._overlap.values():
+            st, code = lynx.lynx_check_error(st_side[0])
+            assert st == lynx.LYNX_OK, (what, st, code)
+        for i, (t, e) in enumerate(zip(sweep.layers, expected)):
+            assert torch.equal(t["Y"].view(torch.int16), e.view(torch.int16)), (what, plan[i][:2])
+
+    for t in sweep.layers:
+        t["Y"].zero_()
+    sweep.run_overlapped(1)
+    check(serial, "overlap eager")
+    for t in sweep.layers:
+        t["Y"].zero_()
+    sweep.capture(overlapped=True, chunks=1)
+    sweep.replay()
+    sweep.replay()
+    check(serial, "overlap graph")
+
+    blocks = []
+    for t in sweep.layers:
+        y = torch.empty_like(t["Y"])
+        for (tt, r0, r1) in sweep.work_items(2):
+            if tt is t:
+                y[r0:r1] = lynx.lynx_linear_act(t["X"][r0:r1], t["W"], t["bias"], t["A"], t["B"],
+                                                skip_sparsify=t["skip"], act=t["act"])
+        blocks.append(y)
+    assert [(r0, r1) for (tt, r0, r1) in sweep.work_items(2) if tt is sweep.layers[0]] == [(0, 256), (256, 384)]
+    for t in sweep.layers:
+        t["Y"].zero_()
+    sweep.run_overlapped(2)
+    check(blocks, "row blocks eager")
+    for t in sweep.layers:
+        t["Y"].zero_()
+    sweep.capture(overlapped=True, chunks=2)
+    sweep.replay()
+    check(blocks, "row blocks graph")
+    sweep.graph = None
