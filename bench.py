@@ -40,8 +40,21 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # capture (dram__bytes_read.sum + dram__bytes_write.sum), with the hash of the
 # GEMM's sources at the capture: the bench reports the figure only while the
 # sources still hash the same, else null ("stale").
-GEMM_SOURCES = ("gemm_pair_kernel.cu", "lynx_ptx.cuh", "lynx_internal.h", "lynx_act.cuh")
-GEMM_DRAM_TRAFFIC = {"mlp_up": {"bytes": 103.165e6 + 82.323e6, "src": "82e9d7345104", "captured": "2026-12-03"}}
+# The sources each kernel's launch depends on (the host code sets its grid and raster).
+KERNEL_SOURCES = {
+    "gemm": ("gemm_pair_kernel.cu", "lynx_ptx.cuh", "lynx_internal.h", "lynx_act.cuh", "lynx_select.cuh",
+             "lynx_api.cu"),
+    "sparsify": ("sparsify_kernel.cu", "lynx_select.cuh", "lynx_ptx.cuh", "lynx_internal.h", "lynx_api.cu"),
+}
+# dram__bytes_read.sum + dram__bytes_write.sum per launch from one ncu capture per
+# workload (profile_layer, L2 flushed before the call), stamped with the hash of
+# the kernel's sources at capture; reported only while the sources still hash so.
+DRAM_TRAFFIC = {
+    "gemm": {"src": "581e8f60d635", "captured": "2026-12-03",
+             "bytes": {"mlp_up": 185362944, "attn_out": 44645888, "mlp_down": 311768320}},
+    "sparsify": {"src": "afb245a4402c", "captured": "2026-12-03",
+                 "bytes": {"mlp_up": 28737792, "attn_out": 25589760, "mlp_down": 148759040}},
+}
 
 def uses_pair_gemm(M, N, K):
     """The library's choice: the CTA-pair GEMM unless the shape cannot feed it."""
@@ -329,6 +342,7 @@ class LayerTimer:
         from activation_sparse_gemm_lynx_b200 import lynx, workloads
 
         self.lynx, self.torch = lynx, torch
+        self.workload, self.act_name = name, act_name
         self.shape = workloads.CONFIGS[name]
         M, N, K, r = self.shape.M, self.shape.N, self.shape.K, self.shape.r
         self.inp = workloads.make_rank_inputs(name, rank)
@@ -418,16 +432,17 @@ def src_hash(files):
     return h.hexdigest()[:12]
 
 
-def stored_gemm_traffic(workload):
-    """ncu's DRAM bytes per launch of the GEMM for this workload, if the stored
-    capture was taken on the GEMM sources as they stand; else (None, why)."""
-    rec = GEMM_DRAM_TRAFFIC.get(workload)
-    if rec is None:
+def stored_traffic(kernel, workload):
+    """ncu's DRAM bytes per launch of `kernel` ("gemm" or "sparsify") on this
+    workload, if the stored capture was taken on the kernel's sources as they
+    stand; else (None, why)."""
+    rec = DRAM_TRAFFIC[kernel]
+    if workload not in rec["bytes"]:
         return None, "not captured for this workload"
-    now = src_hash(GEMM_SOURCES)
+    now = src_hash(KERNEL_SOURCES[kernel])
     if rec["src"] != now:
         return None, f"stale: captured on sources {rec['src']}, kernel now {now}"
-    return rec["bytes"], f"ncu capture of {rec['captured']} (sources {rec['src']})"
+    return rec["bytes"][workload], f"ncu capture of {rec['captured']} (sources {rec['src']})"
 
 
 def layer_summary(lt, ms_linear, parts, dense_ms, peaks, clock_info=None, fused_ms=None):
@@ -442,6 +457,8 @@ def layer_summary(lt, ms_linear, parts, dense_ms, peaks, clock_info=None, fused_
         "sparsify_overhead": max(0.0, 1.0 - parts["gemm_kernel"] / ms_linear),
         "gemm_frac": gemm_tflops / sparse_peak,
         "gemm_tflops": gemm_tflops,
+        "gemm_traffic": stored_traffic("gemm", lt.workload)[0] if lt.act_name == "none" else None,
+        "sparsify_traffic": stored_traffic("sparsify", lt.workload)[0],
         "ms": {"sparsify_kernel": parts["sparsify_kernel"], "gemm_kernel": parts["gemm_kernel"],
                "dense_torch_matmul": dense_ms},
     }
@@ -553,8 +570,9 @@ def run_lynx(args):
     gemm_tflops = flops / (parts["gemm_kernel"] * 1e-3) / 1e12
     sp_bytes = 2 * M * K + M * K + lynx.lynx_meta_bytes(M, K) + 2 * M * r + 4 * M + 2 * r * K
     sp_gbs = sp_bytes / (parts["sparsify_kernel"] * 1e-3) / 1e9
-    traffic, traffic_note = stored_gemm_traffic(args.workload) if act == lynx.LYNX_ACT_NONE \
+    traffic, traffic_note = stored_traffic("gemm", args.workload) if act == lynx.LYNX_ACT_NONE \
         else (None, "not captured with the epilogue activation")
+    sp_traffic, sp_traffic_note = stored_traffic("sparsify", args.workload)
 
     result = {
         "metric": METRIC,
@@ -594,7 +612,7 @@ def run_lynx(args):
         "roofline_sparsify": {
             "bound": "hbm", "kernel": "sparsify_kernel", "achieved": sp_gbs,
             "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": sp_gbs / peaks["hbm_gbs"],
-            "traffic": None,
+            "traffic": sp_traffic, "traffic_note": sp_traffic_note,
             "work": "algorithmic bytes X read 2MK + vals MK + meta MK/8 + T 2Mr + s 4M + A 2rK; "
                     "time: the kernel launched alone",
         },
