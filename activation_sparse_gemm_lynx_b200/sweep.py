@@ -134,6 +134,11 @@ class LinearSweep:
             lynx.lynx_linear_finish(*args, **kw, stream=main)
             done.record(main)
 
+    def side_streams(self):
+        """The side streams the overlapped schedules have used (their sparsify
+        passes report device errors in these streams' status words)."""
+        return [st[0] for st in self._overlap.values()]
+
     def capture(self, overlapped=False, chunks=1):
         """Record one pass into a CUDA graph.  Run the same schedule once first
         (the library's one-time per-device set-up must not happen inside

@@ -776,8 +776,9 @@ def run_sweep(args):
         schedule_ms[name] = max_over_ranks(statistics.mean(timed(g.replay, max(3, min(args.steps, 20)))),
                                            world)
     st, code = lynx.lynx_check_error()
-    if st == lynx.LYNX_OK and sweep._overlap:
-        st, code = lynx.lynx_check_error(next(iter(sweep._overlap.values()))[0])
+    for side in sweep.side_streams():
+        if st == lynx.LYNX_OK:
+            st, code = lynx.lynx_check_error(side)
     if st != lynx.LYNX_OK:
         raise RuntimeError(f"device status after the schedules: {st} code {code:#x}")
     # eager launches (host work in every step) before and after the graph loop

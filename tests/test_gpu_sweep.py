@@ -188,8 +188,8 @@ def test_overlapped_schedules_equal_serial_calls(sweep_and_plan):
         torch.cuda.synchronize()
         st, code = lynx.lynx_check_error()
         assert st == lynx.LYNX_OK, (what, st, code)
-        for st_side in sweep._overlap.values():
-            st, code = lynx.lynx_check_error(st_side[0])
+        for side in sweep.side_streams():
+            st, code = lynx.lynx_check_error(side)
             assert st == lynx.LYNX_OK, (what, st, code)
         for i, (t, e) in enumerate(zip(sweep.layers, expected)):
             assert torch.equal(t["Y"].view(torch.int16), e.view(torch.int16)), (what, plan[i][:2])
