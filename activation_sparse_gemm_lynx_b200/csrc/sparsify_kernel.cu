@@ -391,22 +391,34 @@ sparsify_kernel(const __grid_constant__ SparsifyLaunch p) {
     }
   }
 
-  // ---- T partial of this K range: TMEM -> registers -> global (fp32)
-  if (do_lora && warp >= 2 && warp < 6) {
+  // ---- T partial of this K range: TMEM -> registers -> global (fp32).  The 8
+  // row warps share it: warps w and w + 4 read the same 32 TMEM lanes (rows)
+  // and take alternate 16-column chunks, two chunks per wait.
+  if (do_lora && warp >= 2) {
     const uint32_t row = 32 * (warp & 3) + lane;
     const int64_t grow = mb * 128 + row;
+    const int first = static_cast<int>((warp - 2) >> 2);  // 0 for warps 2-5, 1 for warps 6-9
+    const int chunks = p.r / 16;
     if (!sm.abort_flag && mbar_wait(&sm.tdone, 0)) {
       tc_fence_after();
       float4* dst = reinterpret_cast<float4*>(p.tpart + (static_cast<size_t>(j) * p.M + grow) * p.r);
-      for (int c = 0; c < p.r; c += 16) {
-        uint32_t r[16];
-        tmem_ld_32x32b_x16(sm.tmem_base + ((32u * (warp & 3)) << 16) + static_cast<uint32_t>(c), r);
+      const uint32_t lane_base = sm.tmem_base + ((32u * (warp & 3)) << 16);
+      for (int c = first; c < chunks; c += 4) {
+        const bool two = c + 2 < chunks;
+        uint32_t r[2][16];
+        tmem_ld_32x32b_x16(lane_base + static_cast<uint32_t>(16 * c), r[0]);
+        if (two) tmem_ld_32x32b_x16(lane_base + static_cast<uint32_t>(16 * (c + 2)), r[1]);
         tmem_ld_wait();
         if (grow < p.M) {
 #pragma unroll
-          for (int e = 0; e < 16; e += 4)
-            dst[(c + e) / 4] = make_float4(__uint_as_float(r[e]), __uint_as_float(r[e + 1]),
-                                           __uint_as_float(r[e + 2]), __uint_as_float(r[e + 3]));
+          for (int h = 0; h < 2; ++h) {
+            if (h == 1 && !two) break;
+            const int col = 16 * (c + 2 * h);
+#pragma unroll
+            for (int e = 0; e < 16; e += 4)
+              dst[(col + e) / 4] = make_float4(__uint_as_float(r[h][e]), __uint_as_float(r[h][e + 1]),
+                                               __uint_as_float(r[h][e + 2]), __uint_as_float(r[h][e + 3]));
+          }
         }
       }
       tc_fence_before();
