@@ -52,8 +52,8 @@ KERNEL_SOURCES = {
 DRAM_TRAFFIC = {
     "gemm": {"src": "581e8f60d635", "captured": "2026-12-03",
              "bytes": {"mlp_up": 185362944, "attn_out": 44645888, "mlp_down": 311768320}},
-    "sparsify": {"src": "afb245a4402c", "captured": "2026-12-03",
-                 "bytes": {"mlp_up": 28737792, "attn_out": 25589760, "mlp_down": 148759040}},
+    "sparsify": {"src": "d5bc16ab1aa1", "captured": "2026-12-03",
+                 "bytes": {"mlp_up": 28757504, "attn_out": 25598976, "mlp_down": 149431296}},
 }
 
 def uses_pair_gemm(M, N, K):
