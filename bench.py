@@ -407,7 +407,7 @@ class LayerTimer:
             return tot, first, second
         return tot
 
-    def sparsify_back_to_back(self, reps=8):
+    def sparsify_back_to_back(self, reps=12):
         """Average device time (ms) of one sparsify pass (lynx_linear's first
         kernel alone) launched back to back over distinct copies of X whose
         total exceeds the 126 MB L2 by half again, so that every launch reads
@@ -416,23 +416,24 @@ class LayerTimer:
         torch, lynx = self.torch, self.lynx
         xbytes = self.X.numel() * self.X.element_size()
         copies = [self.X.clone() for _ in range(max(2, -(-(192 << 20) // xbytes)))]
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(reps + 1)]
         lynx.lynx_profile_set_part(1)
         try:
             for x in copies + copies:
                 lynx.lynx_linear(x, self.W, self.bias, self.A, self.B, Y=self.Y, workspace=self.ws)
             self.flush.zero_()
-            e0.record()
-            for _ in range(reps):
+            ev[0].record()
+            for i in range(reps):
                 for x in copies:
                     lynx.lynx_linear(x, self.W, self.bias, self.A, self.B, Y=self.Y, workspace=self.ws)
-            e1.record()
+                ev[i + 1].record()
         finally:
             lynx.lynx_profile_set_part(0)
         torch.cuda.synchronize()
-        launches = reps * len(copies)
+        # the median over the rounds of one launch per copy (a slow round is not averaged in)
+        per_round = [ev[i].elapsed_time(ev[i + 1]) / len(copies) for i in range(reps)]
         del copies
-        return e0.elapsed_time(e1) / launches
+        return statistics.median(per_round)
 
     def parts(self, n):
         """Time of the layer's parts, each run alone (means over n steps):
